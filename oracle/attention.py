@@ -1,0 +1,243 @@
+"""fp64 CPU oracle for exact scaled-dot-product attention (test infrastructure).
+
+THIS IS TEST INFRASTRUCTURE. Only the tests, the smoke check of
+``__graft_entry__`` and the CPU-baseline leg of ``bench.py`` may import it. The
+CUDA path never calls it and shares no code with it.
+
+What it computes follows the FlashAttention pages:
+
+* the definition O = softmax(Q K^T * scale) V of one head (Pranay Mahendrakar,
+  "FlashAttention", Researcher section "The problem being solved"), with the
+  softmax taken safely by subtracting the row maximum (Developer section,
+  "The three running quantities");
+* the per-row statistic the forward pass keeps for the backward pass (paper
+  summary, "Core Idea" item 3, and Researcher section "IO complexity"): the
+  natural-log logsumexp LSE_i = m_i + ln(l_i) of the scaled scores, from which
+  P = exp(S - LSE);
+* the causal flag (Developer section, "Common mistakes": use the flag rather
+  than a dense mask), the 128x128 block-sparse mask (paper summary, "Key Method
+  Details": block-sparse extension) and grouped-query heads (glossary page,
+  "FlashAttention-2 Improvements / Multi-Query Attention Support").
+
+The pages give no backward formulas; the oracle takes the textbook gradient of
+softmax(S) V: dV = P^T dO, dP = dO V^T, D_i = sum_k dO_ik O_ik, dS = P*(dP - D),
+dQ = scale * dS K, dK = scale * dS^T Q, with dK and dV summed over the query
+heads that share a KV head.
+
+Everything is the plain definition: full rows of scores are formed (in row
+chunks only so that memory stays bounded; every row is complete before it is
+normalised). Disallowed pairs are set to -inf; a row with no allowed key gets
+O = 0, LSE = -inf and zero gradients. ``tiled_forward`` restates the pages'
+running-max / running-sum loop separately; it is used only to pin
+``forward`` against the pages' own worked example.
+
+Layouts: Q, dO, O [B, Hq, N, d]; K, V [B, Hkv, N, d]; LSE [B, Hq, N];
+block_mask uint8 [ceil(N/128), ceil(N/128)] shared by every (batch, head).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+BLOCK = 128
+ROW_CHUNK = 512
+
+
+def allowed(rows: np.ndarray, N: int, causal: bool, block_mask) -> np.ndarray:
+    """Boolean [len(rows), N]: key j is visible to query i iff (not causal or
+    j <= i) and (no mask or mask[i // 128, j // 128])."""
+    rows = np.asarray(rows)
+    cols = np.arange(N)
+    ok = np.ones((rows.size, N), dtype=bool)
+    if causal:
+        ok &= cols[None, :] <= rows[:, None]
+    if block_mask is not None:
+        ok &= block_mask[(rows // BLOCK)[:, None], (cols // BLOCK)[None, :]].astype(bool)
+    return ok
+
+
+def softmax_rows(S: np.ndarray):
+    """Safe softmax of each row of S (entries -inf are excluded).
+
+    Returns (P, LSE). Rows that are entirely -inf give P = 0, LSE = -inf.
+    """
+    m = S.max(axis=1)
+    empty = ~np.isfinite(m)
+    m_safe = np.where(empty, 0.0, m)
+    E = np.exp(S - m_safe[:, None])
+    l = E.sum(axis=1)
+    l_safe = np.where(empty, 1.0, l)
+    P = E / l_safe[:, None]
+    lse = np.where(empty, -np.inf, m_safe + np.log(l_safe))
+    return P, lse
+
+
+def _kv_head(h: int, Hq: int, Hkv: int) -> int:
+    return h // (Hq // Hkv)
+
+
+def forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows):
+    """O and LSE of query rows ``rows`` of head (b, h), in fp64."""
+    Hq, Hkv, N = Q.shape[1], K.shape[1], K.shape[2]
+    hk = _kv_head(h, Hq, Hkv)
+    Kh = K[b, hk].astype(np.float64)
+    Vh = V[b, hk].astype(np.float64)
+    rows = np.asarray(rows)
+    O = np.empty((rows.size, Q.shape[3]))
+    L = np.empty(rows.size)
+    for c in range(0, rows.size, ROW_CHUNK):
+        r = rows[c:c + ROW_CHUNK]
+        S = scale * (Q[b, h, r].astype(np.float64) @ Kh.T)
+        S[~allowed(r, N, causal, block_mask)] = -np.inf
+        P, lse = softmax_rows(S)
+        O[c:c + r.size] = P @ Vh
+        L[c:c + r.size] = lse
+    return O, L
+
+
+def forward(Q, K, V, scale, causal=False, block_mask=None):
+    """O [B,Hq,N,d] and LSE [B,Hq,N] in fp64 for all heads."""
+    B, Hq, N, d = Q.shape
+    O = np.empty((B, Hq, N, d))
+    L = np.empty((B, Hq, N))
+    rows = np.arange(N)
+    for b in range(B):
+        for h in range(Hq):
+            O[b, h], L[b, h] = forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows)
+    return O, L
+
+
+def _head_grads(Qh, Kh, Vh, dOh, Oh, scale, causal, block_mask, rows, want_dq=True):
+    """Gradient pieces of one query head restricted to query rows ``rows``.
+
+    Returns (dQ_rows or None, dK contribution [N,d], dV contribution [N,d]).
+    """
+    N = Kh.shape[0]
+    dK = np.zeros_like(Kh)
+    dV = np.zeros_like(Vh)
+    dQ = np.zeros((rows.size, Qh.shape[1])) if want_dq else None
+    for c in range(0, rows.size, ROW_CHUNK):
+        r = rows[c:c + ROW_CHUNK]
+        S = scale * (Qh[r] @ Kh.T)
+        S[~allowed(r, N, causal, block_mask)] = -np.inf
+        P, _ = softmax_rows(S)
+        dP = dOh[r] @ Vh.T
+        D = np.sum(dOh[r] * Oh[r], axis=1)
+        dS = P * (dP - D[:, None])
+        dV += P.T @ dOh[r]
+        dK += scale * (dS.T @ Qh[r])
+        if want_dq:
+            dQ[c:c + r.size] = scale * (dS @ Kh)
+    return dQ, dK, dV
+
+
+def backward(Q, K, V, dO, scale, causal=False, block_mask=None, O=None):
+    """dQ [B,Hq,N,d], dK and dV [B,Hkv,N,d] in fp64.
+
+    O is the oracle's own forward output (recomputed here when not given).
+    """
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    if O is None:
+        O, _ = forward(Q, K, V, scale, causal, block_mask)
+    dQ = np.zeros((B, Hq, N, d))
+    dK = np.zeros((B, Hkv, N, d))
+    dV = np.zeros((B, Hkv, N, d))
+    rows = np.arange(N)
+    for b in range(B):
+        for h in range(Hq):
+            hk = _kv_head(h, Hq, Hkv)
+            dq, dk, dv = _head_grads(Q[b, h].astype(np.float64), K[b, hk].astype(np.float64),
+                                     V[b, hk].astype(np.float64), dO[b, h].astype(np.float64),
+                                     O[b, h], scale, causal, block_mask, rows)
+            dQ[b, h] = dq
+            dK[b, hk] += dk
+            dV[b, hk] += dv
+    return dQ, dK, dV
+
+
+def dq_rows(Q, K, V, dO, scale, causal, block_mask, b, h, rows):
+    """dQ of query rows ``rows`` of head (b, h) (needs only those rows)."""
+    Hq, Hkv = Q.shape[1], K.shape[1]
+    hk = _kv_head(h, Hq, Hkv)
+    rows = np.asarray(rows)
+    O, _ = forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows)
+    Oh = np.zeros((Q.shape[2], Q.shape[3]))
+    Oh[rows] = O
+    dq, _, _ = _head_grads(Q[b, h].astype(np.float64), K[b, hk].astype(np.float64),
+                           V[b, hk].astype(np.float64), dO[b, h].astype(np.float64),
+                           Oh, scale, causal, block_mask, rows)
+    return dq
+
+
+def dkdv_rows(Q, K, V, dO, scale, causal, block_mask, b, hk, key_rows):
+    """dK and dV of key rows ``key_rows`` of KV head (b, hk).
+
+    Every query row that can see one of those keys contributes; for each one
+    the full score row is formed (its LSE and O need all keys).
+    """
+    Hq, Hkv, N = Q.shape[1], K.shape[1], K.shape[2]
+    g = Hq // Hkv
+    key_rows = np.asarray(key_rows)
+    dK = np.zeros((key_rows.size, K.shape[3]))
+    dV = np.zeros((key_rows.size, K.shape[3]))
+    vis = allowed(np.arange(N), N, causal, block_mask)[:, key_rows].any(axis=1)
+    qrows = np.flatnonzero(vis)
+    Kh = K[b, hk].astype(np.float64)
+    Vh = V[b, hk].astype(np.float64)
+    for h in range(hk * g, (hk + 1) * g):
+        Qh = Q[b, h].astype(np.float64)
+        dOh = dO[b, h].astype(np.float64)
+        for c in range(0, qrows.size, ROW_CHUNK):
+            r = qrows[c:c + ROW_CHUNK]
+            S = scale * (Qh[r] @ Kh.T)
+            S[~allowed(r, N, causal, block_mask)] = -np.inf
+            P, _ = softmax_rows(S)
+            O = P @ Vh
+            D = np.sum(dOh[r] * O, axis=1)
+            Pk = P[:, key_rows]
+            dPk = dOh[r] @ Vh[key_rows].T
+            dSk = Pk * (dPk - D[:, None])
+            dV += Pk.T @ dOh[r]
+            dK += scale * (dSk.T @ Qh[r])
+    return dK, dV
+
+
+def tiled_forward(Q2, K2, V2, scale, block, dtype=np.float64, trace=None):
+    """The pages' tiled loop for one head, restated (Developer section, "The
+    algorithm, in plain NumPy"; Researcher section, "Online softmax").
+
+    Key tiles of width ``block`` are visited in order while each query row
+    keeps m (running max), l (running sum of exponentials) and O (running
+    unnormalised output); when a tile raises m, l and O are multiplied by
+    exp(m_old - m_new) before the tile's own terms are added. Returns O / l.
+    All arithmetic is done in ``dtype``. If ``trace`` is a list, the number
+    of rows whose maximum grew is appended for each tile.
+    """
+    Q2 = Q2.astype(dtype)
+    K2 = K2.astype(dtype)
+    V2 = V2.astype(dtype)
+    n = Q2.shape[0]
+    m = np.full(n, -np.inf, dtype=dtype)
+    l = np.zeros(n, dtype=dtype)
+    acc = np.zeros((n, V2.shape[1]), dtype=dtype)
+    sc = dtype(scale)
+    for j0 in range(0, K2.shape[0], block):
+        Sj = (Q2 @ K2[j0:j0 + block].T) * sc
+        m_new = np.maximum(m, Sj.max(axis=1))
+        if trace is not None:
+            trace.append(int(np.count_nonzero(m_new > m)))
+        alpha = np.exp(m - m_new)
+        Pj = np.exp(Sj - m_new[:, None])
+        l = alpha * l + Pj.sum(axis=1)
+        acc = alpha[:, None] * acc + Pj @ V2[j0:j0 + block]
+        m = m_new
+    return acc / l[:, None]
+
+
+def naive_forward_f32(Q2, K2, V2, scale):
+    """The pages' one-shot float32 reference for one head (the N x N score
+    matrix held in full, max-subtracted, exponentiated and normalised)."""
+    S = (Q2.astype(np.float32) @ K2.astype(np.float32).T) * np.float32(scale)
+    S = S - S.max(axis=1, keepdims=True)
+    P = np.exp(S)
+    return (P / P.sum(axis=1, keepdims=True)) @ V2.astype(np.float32)
