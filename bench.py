@@ -1,0 +1,428 @@
+#!/usr/bin/env python
+"""Throughput of exact tiled attention (forward + backward) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step is one pass of the whole hot path over one batch of the workload:
+the fused forward (O and LSE), then the backward's three stages (D / LSE
+preprocess, the dK/dV/dQ kernel, the dQ conversion). The default workload is
+the Llama-7B-shaped causal case (B=4, H=32, N=4096, d=128, bf16), the one the
+forward >= 60% / backward >= 45% of dense-BF16 peak targets are stated on.
+Inputs are seeded synthetic N(0,1) values rounded to bf16; each of Q, K, V, dO
+(134 MB) is larger than the 126 MB L2, so no flush is needed between steps.
+
+Prints one JSON line (rank 0). Under torchrun every rank runs its own copy of
+the workload (independent batches, no collective on the data path: weak
+scaling); the timed region is bracketed by a barrier and a device
+synchronisation on both sides and its duration is the maximum over ranks.
+
+``--impl reference`` times the fp64 CPU oracle instead (the only other
+implementation of this computation here), on the same workload, metric and
+unit, one bounded sample (one batch-head, forward + backward) per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_io_aware_45_b200 import inputs  # noqa: E402
+
+METRIC = "attention fwd+bwd TFLOPS at 1 B200 and % of dense-BF16 tensor peak"
+UNIT = "TFLOP/s"
+FALLBACK_PEAK_TFLOPS = 1590.0
+REASON_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama7b_causal",
+                    choices=[k for k, w in inputs.WORKLOADS.items() if w.backward])
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def workload_config(w: inputs.Workload, world: int) -> dict:
+    return {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} "
+                        f"{'causal' if w.causal else 'non-causal'}"
+                        f"{' block-sparse' if w.sparse else ''} bf16 fwd+bwd",
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
+            "block_sparse": w.sparse, "grad_dtype": "f32",
+            "parallelism": f"replicas x{world} (independent batches)",
+            "l2": "no flush: each of Q, K, V, dO is larger than L2 (126 MB)"
+                  if w.B * w.Hq * w.N * w.d * 2 > 126e6 else "working set may fit L2"}
+
+
+def step_flops(w: inputs.Workload, mask) -> tuple[float, float]:
+    fwd = inputs.flops(w, mask=mask, backward=False)
+    bwd = inputs.flops(w, mask=mask, backward=True)
+    return fwd, bwd
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def oracle_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_sample(w: inputs.Workload, x: dict, b: int, h: int):
+    """Runs the oracle forward + backward of one (batch, query head) and
+    returns (seconds, algorithmic FLOPs of that sample)."""
+    from oracle import attention as orc
+    hk = h // w.group
+    q = x["q"][b:b + 1, h:h + 1]
+    k = x["k"][b:b + 1, hk:hk + 1]
+    v = x["v"][b:b + 1, hk:hk + 1]
+    do = x["do"][b:b + 1, h:h + 1]
+    t0 = time.perf_counter()
+    O, _ = orc.forward(q, k, v, w.scale, w.causal, x["mask"])
+    orc.backward(q, k, v, do, w.scale, w.causal, x["mask"], O=O)
+    dt = time.perf_counter() - t0
+    per = 14.0 * w.d * inputs.allowed_count(w.N, w.causal, x["mask"])
+    return dt, per
+
+
+def cpu_baseline(w, x, budget_s=20.0) -> dict:
+    secs, fl, n = 0.0, 0.0, 0
+    while n == 0 or (secs < budget_s * 0.5 and n < 4):
+        dt, f = oracle_sample(w, x, n % w.B, (n * 7) % w.Hq)
+        secs += dt
+        fl += f
+        n += 1
+    return {"value": fl / secs / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
+            "sample": f"{n} of {w.B * w.Hq} (batch, head) units, forward+backward in fp64 "
+                      f"NumPy ({secs:.1f} s)"}
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    w = inputs.WORKLOADS[args.workload]
+    x = inputs.make_inputs(w)
+    world = int(os.environ.get("WORLD_SIZE", args.gpus))
+    times, fl = [], 0.0
+    for i in range(args.warmup + args.steps):
+        dt, f = oracle_sample(w, x, i % w.B, (i * 7) % w.Hq)
+        if i >= args.warmup:
+            times.append(dt)
+            fl += f
+    total = sum(times)
+    val = fl / total / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(w, world),
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle_threads(),
+                             "kind": "oracle",
+                             "sample": "one (batch, head) unit per step, forward+backward "
+                                       "in fp64 NumPy"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.dev = device_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.out = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "50"],
+                stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.close()
+        sm, smax, reasons = [], [], set()
+        for line in open(self.path):
+            f = [c.strip() for c in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+                mask = int(f[4], 16)
+            except ValueError:
+                continue
+            for bit, name in REASON_BITS.items():
+                if mask & bit and name != "gpu_idle":
+                    reasons.add(name)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- our arm
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        try:
+            return json.load(open(p)), "measured"
+        except Exception:
+            pass
+    return None, "fallback"
+
+
+def traffic_record(kernel_file: str, workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None if the kernel's source changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "exact_io_aware_45_b200", "csrc", kernel_file)
+    if not (os.path.exists(p) and os.path.exists(src)):
+        return None
+    try:
+        recs = json.load(open(p))
+    except Exception:
+        return None
+    sha = hashlib.sha256(open(src, "rb").read()).hexdigest()
+    for r in recs:
+        if r.get("kernel_file") == kernel_file and r.get("source_sha256") == sha and \
+                r.get("workload") == workload:
+            return r.get("dram_bytes_per_launch")
+    return None
+
+
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_45_b200 import fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.lib()
+
+    w = inputs.WORKLOADS[args.workload]
+    x = inputs.make_inputs(w, seed=rank)
+    bf = torch.bfloat16
+    q, k, v, do = (torch.from_numpy(x[n]).to(dev, bf).contiguous() for n in ("q", "k", "v", "do"))
+    mask = None if x["mask"] is None else torch.from_numpy(x["mask"]).to(dev)
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    dq = torch.empty(q.shape, dtype=torch.float32, device=dev)
+    dk = torch.empty(k.shape, dtype=torch.float32, device=dev)
+    dv = torch.empty(v.shape, dtype=torch.float32, device=dev)
+    wsb = fa.fa_bwd_workspace_size(B, Hq, N, d)
+    ws = fa.new_workspace(wsb, dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    P = lambda t: 0 if t is None else t.data_ptr()  # noqa: E731
+    fwd_args = (P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, float(w.scale), int(w.causal),
+                P(mask), fa.FA_BF16, P(ws), sp, fa.PATH_AUTO)
+    bwd_args = (P(q), P(k), P(v), P(o), P(do), P(lse), P(dq), P(dk), P(dv), B, Hq, Hkv, N, d,
+                float(w.scale), int(w.causal), P(mask), fa.FA_BF16, fa.FA_F32, P(ws), wsb, sp,
+                fa.PATH_AUTO)
+    stages = [("fwd", lambda: fa.fa_fwd_ex(*fwd_args)),
+              ("bwd_preprocess", lambda: fa.fa_bwd_preprocess(*bwd_args)),
+              ("bwd_main", lambda: fa.fa_bwd_main(*bwd_args)),
+              ("bwd_finalize", lambda: fa.fa_bwd_finalize(*bwd_args))]
+    n_stage_ev = len(stages) + 1
+
+    def step(evs=None):
+        launches = 0
+        if evs is not None:
+            evs[0].record(stream)
+        for i, (name, fn) in enumerate(stages):
+            s = fn()
+            if s != fa.FA_OK:
+                raise RuntimeError(f"{name}: {fa.status_string(s)}")
+            launches += fa.fa_last_launch_count()
+            if evs is not None:
+                evs[i + 1].record(stream)
+        return launches
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if fa.device_error(ws) != fa.FA_OK:
+        raise RuntimeError("device error word set during warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(n_stage_ev)]
+           for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    launches = 0
+    t_start.record(stream)
+    for i in range(args.steps):
+        launches += step(evs[i])
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    err = fa.device_error(ws)
+    if err != fa.FA_OK:
+        raise RuntimeError(f"device error word set during timing: {fa.status_string(err)}")
+
+    per_stage = {name: statistics.mean(evs[i][j].elapsed_time(evs[i][j + 1])
+                                       for i in range(args.steps))
+                 for j, (name, _) in enumerate(stages)}
+    fwd_fl, bwd_fl = step_flops(w, x["mask"])
+    total_fl = (fwd_fl + bwd_fl) * args.steps * world
+    value = total_fl / (ms / 1e3) / 1e12
+
+    # dominant kernel: the stage with the longest mean duration
+    dom = max(per_stage, key=per_stage.get)
+    dom_fl = {"fwd": fwd_fl, "bwd_main": bwd_fl}.get(dom)
+    peaks, kind = measured_peaks()
+    if dom_fl is not None:
+        peak = (peaks or {}).get("bf16_tflops", FALLBACK_PEAK_TFLOPS)
+        ach = dom_fl / (per_stage[dom] / 1e3) / 1e12
+        kfile = "sm100_fwd.cu" if dom == "fwd" else "sm100_bwd.cu"
+        roof = {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak, "peak_kind": f"{kind} burst bf16",
+                "traffic": traffic_record(kfile, w.name)}
+    else:
+        bytes_ = 4.0 * B * Hq * N * d * 2 + 8.0 * B * Hq * N
+        peak = (peaks or {}).get("hbm_gbs", 6650.0)
+        ach = bytes_ / (per_stage[dom] / 1e3) / 1e9
+        roof = {"bound": "hbm", "kernel": dom, "achieved": ach, "peak": peak, "unit": "GB/s",
+                "frac": ach / peak, "peak_kind": kind, "traffic": None}
+    stage_frac = {}
+    pk = (peaks or {}).get("bf16_tflops", FALLBACK_PEAK_TFLOPS)
+    stage_frac["fwd_tflops"] = fwd_fl / (per_stage["fwd"] / 1e3) / 1e12
+    bwd_ms = per_stage["bwd_preprocess"] + per_stage["bwd_main"] + per_stage["bwd_finalize"]
+    stage_frac["bwd_tflops"] = bwd_fl / (bwd_ms / 1e3) / 1e12
+    stage_frac["fwd_frac_of_peak"] = stage_frac["fwd_tflops"] / pk
+    stage_frac["bwd_frac_of_peak"] = stage_frac["bwd_tflops"] / pk
+
+    # end to end through the C ABI with pinned host buffers
+    e2e = None
+    if args.e2e_steps > 0:
+        hq_, hk_, hv_, hdo = (t.cpu().pin_memory() for t in (q, k, v, do))
+        ho, hl = torch.empty_like(o, device="cpu").pin_memory(), \
+            torch.empty_like(lse, device="cpu").pin_memory()
+        hdq, hdk, hdv = (torch.empty_like(t, device="cpu").pin_memory() for t in (dq, dk, dv))
+        h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (ho, hl, hdq, hdk, hdv))
+
+        def e2e_step():
+            for dst, src in ((q, hq_), (k, hk_), (v, hv_), (do, hdo)):
+                dst.copy_(src, non_blocking=True)
+            s = fa.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, float(w.scale),
+                          int(w.causal), P(mask), fa.FA_BF16, P(ws), sp)
+            if s != fa.FA_OK:
+                raise RuntimeError(fa.status_string(s))
+            s = fa.fa_bwd(*bwd_args[:-1])
+            if s != fa.FA_OK:
+                raise RuntimeError(fa.status_string(s))
+            for dst, src in ((ho, o), (hl, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = a.elapsed_time(b_)
+        if world > 1:
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        e2e = {"value": (fwd_fl + bwd_fl) * args.e2e_steps * world / (ems / 1e3) / 1e12,
+               "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, x)
+
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) rounded to bf16)",
+            "config": workload_config(w, world),
+            "stages_ms": per_stage, "per_direction": stage_frac, "roofline": roof,
+            "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

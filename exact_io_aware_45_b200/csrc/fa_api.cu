@@ -1,0 +1,244 @@
+// C ABI of libfa.so: argument checks, workspace layout, kernel choice.
+//
+// See include/fa.h for the contract. Nothing here allocates device memory;
+// every launch goes to the caller's stream.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include "../../include/fa.h"
+#include "internal.h"
+
+namespace fa {
+
+static thread_local int t_launches = 0;
+void count_launch(int n) { t_launches += n; }
+
+namespace {
+
+constexpr size_t kErrBlock = 256;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool d_supported_simt(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+
+// Common checks of the sizes and flags. Returns FA_OK, or an error code.
+fa_status check_dims(int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                     int dtype) {
+  if (B < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_F32 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (!d_supported_simt(d)) return FA_ERR_UNSUPPORTED;
+  // 64-bit element offsets are used everywhere; keep each tensor under 2^31
+  // rows of d so that row indices fit in int.
+  if ((long long)B * Hq * N >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+void fill_common(Problem& p, int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                 const uint8_t* mask, int dtype, void* stream) {
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.N = N;
+  p.d = d;
+  p.scale = scale;
+  p.causal = causal;
+  p.mask = mask;
+  p.nb = (N + 127) / 128;
+  p.Npad = p.nb * 128;
+  p.dtype = dtype;
+  p.stream = static_cast<cudaStream_t>(stream);
+}
+
+fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_status_string(int s) {
+  switch (s) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED";
+    case FA_ERR_CUDA: return "FA_ERR_CUDA";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_version(void) { return 10000; }
+
+int fa_last_launch_count(void) { return t_launches; }
+
+size_t fa_fwd_workspace_size(void) { return kErrBlock; }
+
+size_t fa_bwd_workspace_size(int B, int Hq, int N, int d) {
+  if (B < 0 || Hq < 0 || N < 0 || d < 0) return 0;
+  const size_t npad = (size_t)((N + 127) / 128) * 128;
+  const size_t vec = align256(sizeof(float) * (size_t)B * Hq * npad);
+  const size_t acc = align256(sizeof(float) * (size_t)B * Hq * N * d);
+  return kErrBlock + 2 * vec + acc;
+}
+
+fa_status fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                    int Hq, int Hkv, int N, int d, float scale, int causal,
+                    const uint8_t* block_mask, int dtype, void* workspace, void* stream,
+                    int path) {
+  t_launches = 0;
+  fa_status s = check_dims(B, Hq, Hkv, N, d, scale, causal, dtype);
+  if (s != FA_OK) return s;
+  if (path != FA_PATH_AUTO && path != FA_PATH_SIMT && path != FA_PATH_TC)
+    return FA_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return FA_OK;
+  if (!Q || !K || !V || !O || !LSE || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) ||
+      !aligned16(workspace))
+    return FA_ERR_INVALID_ARG;
+  Problem p;
+  fill_common(p, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype, stream);
+  p.Q = Q;
+  p.K = K;
+  p.V = V;
+  p.Oout = O;
+  p.LSEout = LSE;
+  p.err = static_cast<unsigned*>(workspace);
+  const bool tc_ok = sm100_fwd_supported(p);
+  if (path == FA_PATH_TC && !tc_ok) return FA_ERR_UNSUPPORTED;
+  const bool use_tc = (path == FA_PATH_TC) || (path == FA_PATH_AUTO && tc_ok);
+  return from_cuda(use_tc ? sm100_fwd(p) : simt_fwd(p));
+}
+
+fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                 int Hq, int Hkv, int N, int d, float scale, int causal,
+                 const uint8_t* block_mask, int dtype, void* workspace, void* stream) {
+  return fa_fwd_ex(Q, K, V, O, LSE, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype,
+                   workspace, stream, FA_PATH_AUTO);
+}
+
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+enum BwdStage { kPre = 1, kMain = 2, kFinal = 4, kAll = 7 };
+
+fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                   const float* LSE, void* dQ, void* dK, void* dV, int B, int Hq, int Hkv,
+                   int N, int d, float scale, int causal, const uint8_t* block_mask, int dtype,
+                   int grad_dtype, void* workspace, size_t workspace_bytes, void* stream,
+                   int path, int stages) {
+  t_launches = 0;
+  fa_status s = check_dims(B, Hq, Hkv, N, d, scale, causal, dtype);
+  if (s != FA_OK) return s;
+  if (grad_dtype != FA_F32 && grad_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (path != FA_PATH_AUTO && path != FA_PATH_SIMT && path != FA_PATH_TC)
+    return FA_ERR_INVALID_ARG;
+  if (B == 0 || N == 0) return FA_OK;
+  if (!Q || !K || !V || !O || !dO || !LSE || !dQ || !dK || !dV || !workspace)
+    return FA_ERR_INVALID_ARG;
+  const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV, workspace};
+  for (const void* q : ptrs)
+    if (!aligned16(q)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_bwd_workspace_size(B, Hq, N, d)) return FA_ERR_INVALID_ARG;
+
+  Problem p;
+  fill_common(p, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype, stream);
+  p.Q = Q;
+  p.K = K;
+  p.V = V;
+  p.O = O;
+  p.dO = dO;
+  p.LSE = LSE;
+  p.dQ = dQ;
+  p.dK = dK;
+  p.dV = dV;
+  p.grad_dtype = grad_dtype;
+  char* ws = static_cast<char*>(workspace);
+  p.err = reinterpret_cast<unsigned*>(ws);
+  const size_t vec = align256(sizeof(float) * (size_t)B * Hq * p.Npad);
+  p.Dws = reinterpret_cast<float*>(ws + kErrBlock);
+  p.LSE2ws = reinterpret_cast<float*>(ws + kErrBlock + vec);
+  p.dQacc = reinterpret_cast<float*>(ws + kErrBlock + 2 * vec);
+
+  const bool tc_ok = sm100_bwd_supported(p);
+  if (path == FA_PATH_TC && !tc_ok) return FA_ERR_UNSUPPORTED;
+  const bool use_tc = (path == FA_PATH_TC) || (path == FA_PATH_AUTO && tc_ok);
+  const bool use_acc = use_tc && sm100_bwd_uses_dq_accumulator(p);
+  cudaError_t e = cudaSuccess;
+  if (stages & kPre) {
+    e = bwd_preprocess(p, use_acc);
+    if (e != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if (stages & kMain) {
+    e = use_tc ? sm100_bwd_main(p) : simt_bwd_main(p);
+    if (e != cudaSuccess) return FA_ERR_CUDA;
+  }
+  if ((stages & kFinal) && use_acc) {
+    e = dq_convert(p);
+    if (e != cudaSuccess) return FA_ERR_CUDA;
+  }
+  return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+fa_status fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                    const float* LSE, void* dQ, void* dK, void* dV, int B, int Hq, int Hkv,
+                    int N, int d, float scale, int causal, const uint8_t* block_mask,
+                    int dtype, int grad_dtype, void* workspace, size_t workspace_bytes,
+                    void* stream, int path) {
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, Hq, Hkv, N, d, scale, causal, block_mask,
+                  dtype, grad_dtype, workspace, workspace_bytes, stream, path, kAll);
+}
+
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                 const float* LSE, void* dQ, void* dK, void* dV, int B, int Hq, int Hkv, int N,
+                 int d, float scale, int causal, const uint8_t* block_mask, int dtype,
+                 int grad_dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, Hq, Hkv, N, d, scale, causal, block_mask,
+                  dtype, grad_dtype, workspace, workspace_bytes, stream, FA_PATH_AUTO, kAll);
+}
+
+#define FA_STAGE_ENTRY(name, stage)                                                            \
+  fa_status name(const void* Q, const void* K, const void* V, const void* O, const void* dO,   \
+                 const float* LSE, void* dQ, void* dK, void* dV, int B, int Hq, int Hkv,       \
+                 int N, int d, float scale, int causal, const uint8_t* block_mask, int dtype,  \
+                 int grad_dtype, void* workspace, size_t workspace_bytes, void* stream,        \
+                 int path) {                                                                   \
+    return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, Hq, Hkv, N, d, scale, causal,          \
+                    block_mask, dtype, grad_dtype, workspace, workspace_bytes, stream, path,   \
+                    stage);                                                                    \
+  }
+
+FA_STAGE_ENTRY(fa_bwd_preprocess, kPre)
+FA_STAGE_ENTRY(fa_bwd_main, kMain)
+FA_STAGE_ENTRY(fa_bwd_finalize, kFinal)
+
+fa_status fa_get_device_error(void* workspace, void* stream) {
+  if (!workspace) return FA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned word = 0;
+  if (cudaMemcpyAsync(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost, st) !=
+      cudaSuccess)
+    return FA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
+  if (word == 0) return FA_OK;
+  if (cudaMemsetAsync(workspace, 0, sizeof(word), st) != cudaSuccess) return FA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FA_ERR_CUDA;
+  return (word & kErrTimeout) ? FA_ERR_TIMEOUT : FA_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// Internal interface between the C ABI (fa_api.cu) and the kernel files.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace fa {
+
+// Everything a launch needs, validated by the ABI layer.
+struct Problem {
+  // inputs
+  const void* Q = nullptr;
+  const void* K = nullptr;
+  const void* V = nullptr;
+  const void* O = nullptr;      // forward output (backward input)
+  const void* dO = nullptr;
+  const float* LSE = nullptr;   // forward LSE (backward input)
+  // outputs
+  void* Oout = nullptr;
+  float* LSEout = nullptr;
+  void* dQ = nullptr;
+  void* dK = nullptr;
+  void* dV = nullptr;
+  // sizes and options
+  int B = 0, Hq = 0, Hkv = 0, N = 0, d = 0;
+  float scale = 1.f;
+  int causal = 0;
+  const uint8_t* mask = nullptr;  // [nb * nb] or null
+  int nb = 0;                     // ceil(N / 128)
+  int dtype = 0;                  // 0 f32, 1 bf16
+  int grad_dtype = 0;
+  // workspace pieces
+  unsigned* err = nullptr;        // device error word
+  float* Dws = nullptr;           // [B*Hq][Npad]
+  float* LSE2ws = nullptr;        // [B*Hq][Npad]  LSE * log2(e), +inf where empty
+  float* dQacc = nullptr;         // [B*Hq][N][d]
+  int Npad = 0;
+  cudaStream_t stream = nullptr;
+};
+
+// Error-word bits set by kernels.
+enum : unsigned { kErrTimeout = 1u, kErrBounds = 2u };
+
+// Counts launches made by the current ABI call (thread-local).
+void count_launch(int n = 1);
+
+// CUDA-core kernels (fp32 arithmetic). simt_kernels.cu
+cudaError_t simt_fwd(const Problem& p);
+cudaError_t bwd_preprocess(const Problem& p, bool zero_dq_accumulator);
+cudaError_t simt_bwd_main(const Problem& p);
+cudaError_t dq_convert(const Problem& p);
+
+// tcgen05 / TMA kernels for sm_100a. sm100_fwd.cu, sm100_bwd.cu
+bool sm100_fwd_supported(const Problem& p);
+cudaError_t sm100_fwd(const Problem& p);
+bool sm100_bwd_supported(const Problem& p);
+bool sm100_bwd_uses_dq_accumulator(const Problem& p);
+cudaError_t sm100_bwd_main(const Problem& p);
+
+}  // namespace fa

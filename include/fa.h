@@ -1,0 +1,173 @@
+/*
+ * fa.h -- C ABI of the exact, IO-aware tiled attention library (libfa.so).
+ *
+ * What is computed (FlashAttention pages: "FlashAttention" lesson by Pranay
+ * Mahendrakar, Researcher section "The problem being solved" and "Online
+ * softmax"; paper summary "FlashAttention: Fast and Memory-Efficient Exact
+ * Attention with IO-Awareness", "Core Idea"):
+ *
+ *   for every batch b and query head h, with KV head hk = h / (Hq / Hkv),
+ *     S   = scale * Q[b,h] K[b,hk]^T                  (N x N, never stored)
+ *     S_ij = -inf where key j is not visible to query i
+ *     O[b,h]   = softmax(S) V[b,hk]                    (row-wise softmax)
+ *     LSE[b,h] = per-row natural-log logsumexp of S    (the saved statistic)
+ *
+ * Key j is visible to query i iff (causal == 0 or j <= i) and (block_mask ==
+ * NULL or block_mask[(i/128) * nb + j/128] != 0), nb = ceil(N/128). A row with
+ * no visible key gets O = 0 and LSE = -inf. The causal flag follows the
+ * lesson's Developer section ("Common mistakes": pass the flag instead of a
+ * dense N x N mask); the 128 x 128 block mask is the block-sparse extension of
+ * the paper summary ("Key Method Details"); grouped KV heads are the
+ * multi-query / grouped-query support of the glossary page ("FlashAttention-2
+ * Improvements").
+ *
+ * The backward pass recomputes P on chip from Q, K and LSE (paper summary,
+ * "Core Idea" item 3) and returns
+ *   dV = P^T dO,  dP = dO V^T,  D_i = sum_k dO_ik O_ik,  dS = P * (dP - D),
+ *   dQ = scale * dS K,  dK = scale * dS^T Q,
+ * with dK and dV summed over the query heads that share a KV head.
+ *
+ * Layout: every tensor is contiguous row-major. Q, O, dO, dQ are [B, Hq, N, d];
+ * K, V, dK, dV are [B, Hkv, N, d]; LSE is float [B, Hq, N]. All tensor
+ * pointers are DEVICE pointers, 16-byte aligned. Outputs are fully
+ * overwritten (dK and dV are not accumulated into). The caller owns every
+ * buffer, including the workspace; the library allocates no device memory.
+ * Every entry point is asynchronous on `stream` (a cudaStream_t passed as
+ * void*; NULL = the legacy default stream) except fa_get_device_error, which
+ * synchronises that stream.
+ *
+ * Errors: argument checks run on the host before any launch and return
+ * FA_ERR_INVALID_ARG (malformed) or FA_ERR_UNSUPPORTED (well-formed but not
+ * implemented: e.g. fp32 inputs with the tensor-core path). A failed launch
+ * returns FA_ERR_CUDA. Every wait inside a kernel is bounded; a wait that runs
+ * out sets a bit in the workspace's error word, the kernel returns without
+ * faulting, and fa_get_device_error reports FA_ERR_TIMEOUT. The library never
+ * traps and never resets the device.
+ */
+#ifndef FA_H_
+#define FA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,
+  FA_ERR_UNSUPPORTED = 2,
+  FA_ERR_CUDA = 3,
+  FA_ERR_TIMEOUT = 4
+} fa_status;
+
+/* Element types of Q, K, V, O, dO (dtype) and of dQ, dK, dV (grad_dtype). */
+typedef enum { FA_F32 = 0, FA_BF16 = 1 } fa_dtype;
+
+/* Kernel family: AUTO picks the tcgen05 tensor-core kernels for bf16 with
+ * d in {64, 128} and the fp32 CUDA-core kernels otherwise; SIMT forces the
+ * CUDA-core kernels (fp32 arithmetic for any supported dtype); TC forces the
+ * tensor-core kernels (FA_ERR_UNSUPPORTED where they do not apply). */
+typedef enum { FA_PATH_AUTO = 0, FA_PATH_SIMT = 1, FA_PATH_TC = 2 } fa_path;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(int status);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int fa_version(void);
+
+/* Bytes of workspace fa_fwd needs: the 256-byte error-word block. */
+size_t fa_fwd_workspace_size(void);
+
+/* Bytes of workspace fa_bwd needs: the error-word block, D and the
+ * log2-scaled LSE (float [B*Hq][ceil(N/128)*128] each) and the fp32 dQ
+ * accumulator (float [B*Hq][N][d]). Returns 0 for negative sizes. */
+size_t fa_bwd_workspace_size(int B, int Hq, int N, int d);
+
+/*
+ * Forward pass. Writes O (dtype) and LSE (float, natural log of the scaled
+ * scores, -inf for rows with no visible key).
+ *   Q [B,Hq,N,d], K and V [B,Hkv,N,d] (dtype); O [B,Hq,N,d] (dtype);
+ *   LSE [B,Hq,N] float; scale: the softmax scale (1/sqrt(d) in the pages);
+ *   causal: 0 or 1; block_mask: NULL or device uint8 [nb*nb];
+ *   workspace: >= fa_fwd_workspace_size() bytes, device, zeroed once before
+ *   first use (it then holds the error word, which fa_get_device_error clears).
+ * Supported: d in {16, 32, 64, 128}; Hq % Hkv == 0; N >= 0, B >= 0 (an empty
+ * problem launches nothing and returns FA_OK).
+ */
+fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                 int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                 const uint8_t* block_mask, int dtype, void* workspace, void* stream);
+
+/* fa_fwd with an explicit kernel family (fa_path). */
+fa_status fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                    int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                    const uint8_t* block_mask, int dtype, void* workspace, void* stream,
+                    int path);
+
+/*
+ * Backward pass: dQ, dK, dV (grad_dtype) from Q, K, V, O, dO (dtype) and the
+ * forward's LSE. scale, causal and block_mask must be the forward's.
+ * workspace: >= fa_bwd_workspace_size(B, Hq, N, d) bytes of device memory
+ * (error word zeroed once before first use; the rest is scratch, overwritten).
+ * Runs three stages in order on `stream`: fa_bwd_preprocess, fa_bwd_main,
+ * fa_bwd_finalize.
+ */
+fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                 const float* LSE, void* dQ, void* dK, void* dV,
+                 int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                 const uint8_t* block_mask, int dtype, int grad_dtype,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* fa_bwd with an explicit kernel family (fa_path). */
+fa_status fa_bwd_ex(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                    const float* LSE, void* dQ, void* dK, void* dV,
+                    int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                    const uint8_t* block_mask, int dtype, int grad_dtype,
+                    void* workspace, size_t workspace_bytes, void* stream, int path);
+
+/*
+ * The three stages of fa_bwd, exposed so that each kernel can be timed on
+ * its own. They take fa_bwd_ex's arguments and must be called in this order
+ * with the same arguments and workspace.
+ *   preprocess: D_i = sum_k dO_ik O_ik and LSE * log2(e) into the workspace
+ *               (rows with LSE = -inf become +inf, so their P is 0); zeroes
+ *               the dQ accumulator when the main stage uses one.
+ *   main:       recomputes P tile by tile; writes dK, dV and accumulates dQ.
+ *   finalize:   converts the fp32 dQ accumulator to dQ (no launch when the
+ *               main stage wrote dQ directly).
+ */
+fa_status fa_bwd_preprocess(const void* Q, const void* K, const void* V, const void* O,
+                            const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                            int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                            const uint8_t* block_mask, int dtype, int grad_dtype,
+                            void* workspace, size_t workspace_bytes, void* stream, int path);
+fa_status fa_bwd_main(const void* Q, const void* K, const void* V, const void* O,
+                      const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                      int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                      const uint8_t* block_mask, int dtype, int grad_dtype,
+                      void* workspace, size_t workspace_bytes, void* stream, int path);
+fa_status fa_bwd_finalize(const void* Q, const void* K, const void* V, const void* O,
+                          const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                          int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                          const uint8_t* block_mask, int dtype, int grad_dtype,
+                          void* workspace, size_t workspace_bytes, void* stream, int path);
+
+/* Number of kernel launches the last successful call of fa_fwd_ex / fa_bwd_ex
+ * or one of the stages made from the calling thread (for launch accounting). */
+int fa_last_launch_count(void);
+
+/*
+ * Reads and clears the workspace's error word: synchronises `stream`, copies
+ * the word to the host, then zeroes it. Returns FA_OK if no kernel recorded a
+ * failure, FA_ERR_TIMEOUT if a bounded wait ran out, FA_ERR_CUDA if the copy
+ * failed (and then leaves the word as it is).
+ */
+fa_status fa_get_device_error(void* workspace, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_H_ */
