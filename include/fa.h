@@ -154,6 +154,41 @@ fa_status fa_bwd_finalize(const void* Q, const void* K, const void* V, const voi
                           const uint8_t* block_mask, int dtype, int grad_dtype,
                           void* workspace, size_t workspace_bytes, void* stream, int path);
 
+/*
+ * fa_bwd_noalloc -- the backward pass for callers that cannot allocate.
+ *
+ * No passage of the FlashAttention pages corresponds to this entry point; it
+ * exists for deployment. Some callers cannot call cudaMalloc or provide a
+ * workspace buffer: code running under an allocator that owns all device
+ * memory and forbids side allocations, plugins whose host hands them only
+ * the tensors, or paths where an allocation could block or fragment a
+ * memory pool. This entry point computes what fa_bwd computes with fp32
+ * gradients (same kernels), but its scratch -- the per-row D = rowsum(dO * O)
+ * and LSE * log2(e) vectors -- lives in a fixed array inside libfa.so's
+ * device image (about 8 MiB, held by every GPU that loads the library until
+ * the process exits). It allocates nothing and calls no allocating routine.
+ *
+ * Arguments as fa_bwd, except: dQ, dK, dV are float (fp32 gradients only);
+ * there is no workspace; device_error is NULL or a caller-owned device word
+ * (4-byte aligned) into which kernels OR a non-zero value if a bounded wait
+ * runs out (the caller zeroes it; with NULL a word inside the fixed array is
+ * used and cleared at each call, so timeouts are then not observable).
+ *
+ * Limits: B * Hq * ceil(N / 128) * 128 must not exceed 1,048,576 rows
+ * (FA_ERR_UNSUPPORTED otherwise, before anything is launched).
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any CUDA graph
+ * capture. Every call on a device shares the one array and leaves its
+ * contents behind; calls whose kernels overlap on the GPU (different streams
+ * without ordering, or several host threads) race on it and must be ordered
+ * by the caller.
+ */
+fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void* O,
+                         const void* dO, const float* LSE, float* dQ, float* dK, float* dV,
+                         int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                         const uint8_t* block_mask, int dtype, unsigned* device_error,
+                         void* stream);
+
 /* Number of kernel launches the last successful call of fa_fwd_ex / fa_bwd_ex
  * or one of the stages made from the calling thread (for launch accounting). */
 int fa_last_launch_count(void);
