@@ -1,6 +1,419 @@
-// Placeholder: the tcgen05 forward is not enabled yet.
-#include "internal.h"
+// Fused attention forward for sm_100a: tcgen05 MMAs with TMEM accumulators,
+// TMA-fed K/V ring, warp-specialised producer / MMA / softmax warps.
+//
+// Computes, for each query row, O = softmax(scale * Q K^T) V over the visible
+// keys and LSE = logsumexp(scale * Q K^T) (FlashAttention lesson, Researcher
+// section "The problem being solved"), never writing S or P to HBM (paper
+// summary, "Core Idea" items 1, 2 and 4). Each CTA owns two 128-row query tiles
+// of one (batch, head) and walks the key tiles both need; for each key tile j:
+//
+//   S_t = Q_t K_j^T             tcgen05.mma, A and B from shared memory, S in TMEM
+//   online softmax on S_t       one thread per row (tcgen05.ld 32x32b), base-2
+//                               exponentials with scale*log2(e) folded in
+//   O_t += P_t V_j              tcgen05.mma, P (bf16) from TMEM, V from shared memory
+//
+// The running statistics follow the Researcher section's "Online softmax"
+// recurrence: m^(j) = max(m^(j-1), rowmax S^(j)), l^(j) = e^(m^(j-1)-m^(j))
+// l^(j-1) + rowsum e^(S^(j)-m^(j)), and O^(j) likewise. The kernel keeps a
+// reference maximum per row and moves it (rescaling l and the TMEM
+// accumulator together, the "correction" step) only when a tile's row maximum
+// exceeds it by more than 2^8 in the exponent; between moves the terms are
+// taken relative to the unchanged reference. The recurrence holds for any
+// reference value, so O^(T)/l^(T) is unchanged; the bound keeps every P term
+// <= 256 (no overflow in fp32 or bf16) and skips most TMEM round trips.
+//
+// Two query tiles alternate on the tensor core (ping-pong): while one
+// softmax warpgroup works on S_0, the MMA warp runs P_1 V and Q_1 K^T, and the
+// other way round. P_t is written into the upper half of S_t's TMEM columns;
+// tcgen05.mma operations issued by one thread execute in order, so the next
+// Q_t K^T that overwrites S_t cannot overtake the P_t V that reads it.
+//
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
+// TMEM allocator, warp 3 builds the key-tile list, warps 4-7 softmax of query
+// tile 0, warps 8-11 softmax of query tile 1.
+#include <math.h>
+
+#include "sm100_common.cuh"
+
 namespace fa {
-bool sm100_fwd_supported(const Problem&) { return false; }
-cudaError_t sm100_fwd(const Problem&) { return cudaErrorNotSupported; }
+namespace {
+using namespace sm100;
+
+constexpr int kBM = 128;           // query rows per tile
+constexpr int kBN = 128;           // keys per tile
+constexpr int kMaxTiles = 2048;    // key tiles per sequence: N <= 262144
+constexpr int kThreads = 384;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kTau = 8.0f;       // reference-max slack, log2 units
+
+template <int D>
+struct Cfg {
+  static constexpr int kStages = (D == 64) ? 4 : 2;
+  static constexpr int kTileBytes = kBN * D * 2;   // one K or V tile (bf16)
+  static constexpr int kQBytes = kBM * D * 2;
+  static constexpr int kColBlocks = D / 64;        // 128-byte column blocks per row
+  static constexpr int kBlockBytes = 128 * 128;    // one column block of a 128-row tile
+  static constexpr uint32_t kS0 = 0, kS1 = 128;
+  static constexpr uint32_t kO0 = 256, kO1 = 256 + (D == 64 ? 64 : 128);
+  static constexpr uint32_t kPOff = 64;            // P (bf16 pairs) inside S's columns
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + 2 * kQBytes;
+  static constexpr int kOffV = kOffK + kStages * kTileBytes;
+  static constexpr int kOffEnd = kOffV + kStages * kTileBytes;
+};
+
+struct alignas(16) Ctl {
+  uint64_t q_full;
+  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint64_t s_full[2], p_full[2];
+  uint64_t o_done;
+  uint32_t tmem_base;
+  int abort;
+  int ntiles;
+  uint16_t tiles[kMaxTiles];
+  uint8_t dead[kMaxTiles];   // bit t: query tile t sees nothing of this key tile
+};
+
+struct FwdParams {
+  CUtensorMap tq, tk, tv;    // [B*H][N][d] bf16, box {64, 128, 1}, 128B swizzle
+  __nv_bfloat16* O;
+  float* LSE;
+  const uint8_t* mask;
+  unsigned* err;
+  int N, Hq, Hkv, nb, nblk, causal;
+  float c;                   // scale * log2(e)
+};
+
+// Bounded wait that ignores the abort flag (used only to drain in-flight work).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) break;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
+  using C = Cfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem_raw);
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t tile_addr = (raw_addr + sizeof(Ctl) + 1023u) & ~1023u;
+  uint8_t* tiles_base = smem_raw + (tile_addr - raw_addr);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bh = blockIdx.x;                     // b * Hq + h
+  const int blk = p.nblk - 1 - blockIdx.y;       // longest causal rows first
+  const int h = bh % p.Hq, b = bh / p.Hq;
+  const int bhk = b * p.Hkv + h / (p.Hq / p.Hkv);
+  const int q0 = blk * 2 * kBM;
+  const int qb0 = 2 * blk, qb1 = 2 * blk + 1;   // 128-row mask blocks of the two tiles
+  const int N = p.N;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctl.q_full, 1);
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&ctl.k_full[s], 1);
+      mbar_init(&ctl.v_full[s], 1);
+      mbar_init(&ctl.kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctl.s_full[t], 1);
+      mbar_init(&ctl.p_full[t], 4);
+    }
+    mbar_init(&ctl.o_done, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&ctl.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 3) {
+    // Key tiles either query tile can see, in increasing order.
+    const int kb_end = p.causal ? min(p.nb, qb1 + 1) : p.nb;
+    int count = 0;
+    for (int kb0 = 0; kb0 < kb_end; kb0 += 32) {
+      const int kb = kb0 + lane;
+      bool a0 = false, a1 = false;
+      if (kb < kb_end) {
+        a0 = (!p.mask || p.mask[(size_t)qb0 * p.nb + kb]) && (!p.causal || kb <= qb0);
+        a1 = qb1 < p.nb && (!p.mask || p.mask[(size_t)qb1 * p.nb + kb]) &&
+             (!p.causal || kb <= qb1);
+      }
+      const bool act = a0 || a1;
+      const unsigned bal = __ballot_sync(0xffffffffu, act);
+      if (act) {
+        const int pos = count + __popc(bal & ((1u << lane) - 1u));
+        ctl.tiles[pos] = static_cast<uint16_t>(kb);
+        ctl.dead[pos] = static_cast<uint8_t>((a0 ? 0 : 1) | (a1 ? 0 : 2));
+      }
+      count += __popc(bal);
+    }
+    if (lane == 0) ctl.ntiles = count;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = ctl.tmem_base;
+  const int T = ctl.ntiles;
+  const Guard g{&ctl.abort, p.err};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && T > 0) {
+      prefetch_tmap(&p.tq);
+      prefetch_tmap(&p.tk);
+      prefetch_tmap(&p.tv);
+      mbar_expect_tx(&ctl.q_full, 2 * C::kQBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_load_3d(tiles_base + C::kOffQ + t * C::kQBytes + cb * C::kBlockBytes, &p.tq,
+                      &ctl.q_full, cb * 64, q0 + t * kBM, bh);
+      int issued = 0;
+      for (int j = 0; j < T; ++j) {
+        const int s = j % C::kStages;
+        if (j >= C::kStages && !mbar_wait(&ctl.kv_empty[s], ((j / C::kStages) - 1) & 1, g))
+          break;
+        const int kb = ctl.tiles[j];
+        mbar_expect_tx(&ctl.k_full[s], C::kTileBytes);
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_load_3d(tiles_base + C::kOffK + s * C::kTileBytes + cb * C::kBlockBytes, &p.tk,
+                      &ctl.k_full[s], cb * 64, kb * kBN, bhk);
+        mbar_expect_tx(&ctl.v_full[s], C::kTileBytes);
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_load_3d(tiles_base + C::kOffV + s * C::kTileBytes + cb * C::kBlockBytes, &p.tv,
+                      &ctl.v_full[s], cb * 64, kb * kBN, bhk);
+        issued = j + 1;
+      }
+      // Every issued copy has landed before the CTA may exit.
+      drain_wait(&ctl.q_full, 0);
+      for (int s = 0; s < C::kStages && s < issued; ++s) {
+        const int n_s = (issued - 1 - s) / C::kStages + 1;  // loads into stage s
+        drain_wait(&ctl.k_full[s], (n_s - 1) & 1);
+        drain_wait(&ctl.v_full[s], (n_s - 1) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t idS = idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t idO = idesc_bf16(kBM, D, false, true);
+      const uint32_t qa = smem_u32(tiles_base + C::kOffQ);
+      const uint32_t ka = smem_u32(tiles_base + C::kOffK);
+      const uint32_t va = smem_u32(tiles_base + C::kOffV);
+      auto issue_s = [&](int t, int stage) {
+        const uint32_t qt = qa + t * C::kQBytes, kt = ka + stage * C::kTileBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          mma_ss(tm + (t ? C::kS1 : C::kS0), sdesc_sw128(qt + off, 16, 1024),
+                 sdesc_sw128(kt + off, 16, 1024), idS, kk > 0);
+        }
+      };
+      auto issue_pv = [&](int t, int stage, bool acc) {
+        const uint32_t vt = va + stage * C::kTileBytes;
+        const uint32_t pt = tm + (t ? C::kS1 : C::kS0) + C::kPOff;
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk)
+          mma_ts(tm + (t ? C::kO1 : C::kO0), pt + kk * 8,
+                 sdesc_sw128(vt + kk * 16 * 128, C::kBlockBytes, 1024), idO, (acc || kk > 0));
+      };
+      bool ok = mbar_wait(&ctl.q_full, 0, g) && mbar_wait(&ctl.k_full[0], 0, g);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        mma_commit(&ctl.s_full[0]);
+        issue_s(1, 0);
+        mma_commit(&ctl.s_full[1]);
+      }
+      for (int j = 0; ok && j < T; ++j) {
+        const int s = j % C::kStages;
+        const uint32_t ph = (j / C::kStages) & 1;
+        if (!(ok = mbar_wait(&ctl.v_full[s], ph, g) && mbar_wait(&ctl.p_full[0], j & 1, g)))
+          break;
+        tc_fence_after();
+        issue_pv(0, s, j > 0);
+        const bool more = j + 1 < T;
+        const int s2 = (j + 1) % C::kStages;
+        if (more) {
+          if (!(ok = mbar_wait(&ctl.k_full[s2], ((j + 1) / C::kStages) & 1, g))) break;
+          tc_fence_after();
+          issue_s(0, s2);
+          mma_commit(&ctl.s_full[0]);
+        }
+        if (!(ok = mbar_wait(&ctl.p_full[1], j & 1, g))) break;
+        tc_fence_after();
+        issue_pv(1, s, j > 0);
+        mma_commit(&ctl.kv_empty[s]);
+        if (more) {
+          issue_s(1, s2);
+          mma_commit(&ctl.s_full[1]);
+        }
+      }
+      mma_commit(&ctl.o_done);
+      drain_wait(&ctl.o_done, 0);   // no MMA may still run when TMEM is freed
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax
+    const int t = (warp - 4) >> 2;           // query tile of this warpgroup
+    const int wq = warp & 3;                 // TMEM lane quarter of this warp
+    const int r = wq * 32 + lane;            // row inside the tile
+    const int row = q0 + t * kBM + r;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t sreg = tm + (t ? C::kS1 : C::kS0) + lane_off;
+    const uint32_t oreg = tm + (t ? C::kO1 : C::kO0) + lane_off;
+    const float c = p.c;
+    const int tile_row0 = q0 + t * kBM;
+    float m_ref = -INFINITY, l = 0.f;
+    for (int j = 0; j < T; ++j) {
+      if (!mbar_wait(&ctl.s_full[t], j & 1, g)) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld64(sreg, *reinterpret_cast<uint32_t(*)[64]>(&sr[0]));
+      tmem_ld64(sreg + 64, *reinterpret_cast<uint32_t(*)[64]>(&sr[64]));
+      const int col0 = ctl.tiles[j] * kBN;
+      const bool dead = (ctl.dead[j] >> t) & 1;
+      const bool need_mask = dead || col0 + kBN > N || (p.causal && col0 + kBN - 1 > tile_row0);
+      float mx = -INFINITY;
+      if (need_mask) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) {
+          const int col = col0 + i;
+          const bool bad = dead || col >= N || (p.causal && col > row);
+          const float v = bad ? -INFINITY : __uint_as_float(sr[i]);
+          sr[i] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
+      }
+      const float mx2 = mx * c;
+      const bool grow = mx2 > m_ref + kTau;
+      float alpha = 1.f;
+      if (grow) {
+        alpha = ex2(m_ref - mx2);   // 0 when there was no reference yet
+        m_ref = mx2;
+        l *= alpha;
+      }
+      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+      uint32_t pk[64];
+      float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        const float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), c, -mu));
+        const float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), c, -mu));
+        sum0 += p0;
+        sum1 += p1;
+        pk[i] = pack_bf16(p0, p1);
+      }
+      l += sum0 + sum1;
+      // The accumulator holds P V of earlier tiles (complete: the commit that
+      // signalled S_t came after them); rescale it where the reference moved.
+      if (__any_sync(0xffffffffu, grow && j > 0)) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(oreg + cc * 32, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(oreg + cc * 32, o);
+        }
+      }
+      tmem_st32(sreg + C::kPOff, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(sreg + C::kPOff + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.p_full[t]);
+    }
+    // ------------------------------------------------------------ epilogue
+    if (T > 0) {
+      mbar_wait(&ctl.o_done, 0, g);
+      tc_fence_after();
+    }
+    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+    const bool valid = row < N;
+    __nv_bfloat16* out = p.O + ((size_t)bh * N + (valid ? row : 0)) * D;
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      if (T > 0) {
+        tmem_ld32(oreg + cc * 32, o);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o[i] = 0u;
+      }
+      uint4 v[4];
+      uint32_t* vw = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        vw[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+      if (valid) {
+        uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dst[i] = v[i];
+      }
+    }
+    if (valid) p.LSE[(size_t)bh * N + row] = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tm, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch(const Problem& pr) {
+  using C = Cfg<D>;
+  FwdParams kp;
+  memset(&kp, 0, sizeof(kp));
+  const uint64_t BHq = (uint64_t)pr.B * pr.Hq, BHk = (uint64_t)pr.B * pr.Hkv;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_tmap_3d(&kp.tq, pr.Q, bf, 2, D, pr.N, BHq, 64, kBM, sw) ||
+      !make_tmap_3d(&kp.tk, pr.K, bf, 2, D, pr.N, BHk, 64, kBN, sw) ||
+      !make_tmap_3d(&kp.tv, pr.V, bf, 2, D, pr.N, BHk, 64, kBN, sw))
+    return cudaErrorInvalidValue;
+  kp.O = static_cast<__nv_bfloat16*>(pr.Oout);
+  kp.LSE = pr.LSEout;
+  kp.mask = pr.mask;
+  kp.err = pr.err;
+  kp.N = pr.N;
+  kp.Hq = pr.Hq;
+  kp.Hkv = pr.Hkv;
+  kp.nb = pr.nb;
+  kp.nblk = (pr.N + 2 * kBM - 1) / (2 * kBM);
+  kp.causal = pr.causal;
+  kp.c = pr.scale * kLog2e;
+  const size_t smem = sizeof(Ctl) + 1024 + C::kOffEnd;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  dim3 grid((unsigned)BHq, (unsigned)kp.nblk);
+  fwd_kernel<D><<<grid, kThreads, smem, pr.stream>>>(kp);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sm100_fwd_supported(const Problem& p) {
+  return p.dtype == 1 && (p.d == 64 || p.d == 128) && p.scale > 0.f && p.nb <= kMaxTiles &&
+         (long long)p.B * p.Hq < (1ll << 31);
+}
+
+cudaError_t sm100_fwd(const Problem& p) {
+  return p.d == 64 ? launch<64>(p) : launch<128>(p);
+}
+
 }  // namespace fa
