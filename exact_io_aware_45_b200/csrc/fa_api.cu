@@ -173,10 +173,14 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   const bool tc_ok = sm100_bwd_supported(p);
   if (path == FA_PATH_TC && !tc_ok) return FA_ERR_UNSUPPORTED;
   const bool use_tc = (path == FA_PATH_TC) || (path == FA_PATH_AUTO && tc_ok);
+  // The tensor-core path accumulates dQ in fp32: straight into dQ for fp32
+  // gradients, into the workspace accumulator (converted by the finalize
+  // stage) for bf16 gradients. The preprocess zeroes whichever it is.
   const bool use_acc = use_tc && sm100_bwd_uses_dq_accumulator(p);
+  if (use_tc && !use_acc) p.dQacc = static_cast<float*>(dQ);
   cudaError_t e = cudaSuccess;
   if (stages & kPre) {
-    e = bwd_preprocess(p, use_acc);
+    e = bwd_preprocess(p, use_tc);
     if (e != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stages & kMain) {

@@ -1,7 +1,495 @@
-// Placeholder: the tcgen05 backward is not built yet.
-#include "internal.h"
+// Attention backward for sm_100a: one CTA per 128-key tile of one (batch, KV
+// head), tcgen05 MMAs with dK and dV accumulated in TMEM for the whole CTA,
+// P recomputed on chip from Q, K and the forward's LSE (paper summary, "Core
+// Idea" item 3: recomputation instead of storing the N x N matrix).
+//
+// For each visible (query head of the KV group, query tile) item i:
+//
+//   S^T  = K Q_i^T                 SS MMA -> TMEM
+//   dP^T = V dO_i^T                SS MMA -> TMEM
+//   P^T  = exp2(S^T * scale*log2e - LSE2_i)      softmax warps, one key row per thread
+//   dS^T = P^T * (dP^T - D_i)                    (D_i = rowsum(dO_i * O_i), preprocess)
+//   dV  += P^T dO_i                TS MMA (P^T bf16 in TMEM)
+//   dK  += dS^T Q_i                SS MMA (dS^T bf16 in shared memory)
+//   dQ_i = dS_i K   (d = 64)  or  dQ_i^T = K^T dS_i^T   (d = 128)   SS MMA -> TMEM
+//   dQ accumulator += scale * dQ_i  TMA reduce-add from shared memory
+//
+// Query tiles are 128 rows for d = 64 and 64 rows for d = 128 so that every
+// accumulator fits the 512 TMEM columns; the dQ product is arranged so its
+// M dimension is 128 either way.
+//
+// MMA issue order per item: dV(i), S(i+1), dP(i+1), dK(i), dQ(i). tcgen05.mma
+// operations from one thread run in order, so the softmax of item i+1 (which
+// waits for S(i+1)/dP(i+1)) knows dV(i) has read P^T(i) from the S columns it
+// overwrites, and that item i-1's dK/dQ have read the dS^T buffer it reuses
+// (double-buffered by item parity).
+//
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
+// TMEM allocator, warp 3 builds the query-tile list, warps 4-7 softmax / dS
+// and the dK, dV epilogue, warps 8-11 drain dQ from TMEM to the global fp32
+// accumulator.
+#include <math.h>
+
+#include <algorithm>
+
+#include "sm100_common.cuh"
+
 namespace fa {
-bool sm100_bwd_supported(const Problem&) { return false; }
-bool sm100_bwd_uses_dq_accumulator(const Problem&) { return false; }
-cudaError_t sm100_bwd_main(const Problem&) { return cudaErrorNotSupported; }
+namespace {
+using namespace sm100;
+
+constexpr int kBN = 128;            // keys per CTA
+constexpr int kMaxQTiles = 4096;    // query tiles per sequence
+constexpr int kThreads = 384;
+constexpr int kStages = 2;          // Q / dO ring depth
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct Cfg {
+  static constexpr int MQ = (D == 64) ? 128 : 64;         // query rows per item
+  static constexpr int kKVBytes = kBN * D * 2;            // K or V tile
+  static constexpr int kQBytes = MQ * D * 2;              // Q or dO tile
+  static constexpr int kQBlock = MQ * 128;                // one 64-column block of Q / dO
+  static constexpr int kDSBytes = kBN * MQ * 2;           // dS^T buffer (bf16)
+  static constexpr int kStgBytes = MQ * D * 4;            // dQ staging (fp32)
+  static constexpr int kStgBox = MQ * 128;                // one 32-column fp32 box
+  // TMEM columns
+  static constexpr uint32_t kDK = 0, kDV = D, kS = 2 * D, kDP = 2 * D + MQ,
+                            kDQ = 2 * D + 2 * MQ;
+  // shared memory (offsets from a 1024-aligned base)
+  static constexpr int kOffK = 0;
+  static constexpr int kOffV = kOffK + kKVBytes;
+  static constexpr int kOffQ = kOffV + kKVBytes;
+  static constexpr int kOffDO = kOffQ + kStages * kQBytes;
+  static constexpr int kOffDS = kOffDO + kStages * kQBytes;
+  static constexpr int kOffStg = kOffDS + 2 * kDSBytes;
+  static constexpr int kOffVec = kOffStg + kStgBytes;       // [stage][LSE2 | D][MQ] floats
+  static constexpr int kOffEnd = kOffVec + kStages * 2 * MQ * 4;
+  static_assert(kDQ + 64 <= 512, "TMEM budget");
+};
+
+struct alignas(16) Ctl {
+  uint64_t kv_full;
+  uint64_t qdo_full[kStages], qdo_empty[kStages];
+  uint64_t sp_full, p_ready, dq_full, dq_free, acc_done;
+  uint32_t tmem_base;
+  int abort;
+  int nq;                      // visible query tiles per query head
+  uint16_t qtiles[kMaxQTiles];
+};
+
+struct BwdParams {
+  CUtensorMap tq, tdo;         // [B*Hq][N][d] bf16, box {64, MQ}, 128B swizzle
+  CUtensorMap tk, tv;          // [B*Hkv][N][d] bf16, box {64, 128}
+  CUtensorMap tdq;             // [B*Hq][N][d] fp32, box {32, MQ}, 128B swizzle (reduce-add)
+  const float* lse2;           // [B*Hq][Npad]
+  const float* dvec;           // [B*Hq][Npad]
+  void* dK;
+  void* dV;
+  const uint8_t* mask;
+  unsigned* err;
+  int N, Npad, Hq, Hkv, nb, causal, grad_bf16, BHk;
+  float c;                     // scale * log2(e)
+  float scale;
+};
+
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitLimitCycles) break;
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
+  using C = Cfg<D>;
+  constexpr int MQ = C::MQ;
+  extern __shared__ uint8_t smem_raw[];
+  Ctl& ctl = *reinterpret_cast<Ctl*>(smem_raw);
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t base_addr = (raw_addr + sizeof(Ctl) + 1023u) & ~1023u;
+  uint8_t* base = smem_raw + (base_addr - raw_addr);
+  float* vec = reinterpret_cast<float*>(base + C::kOffVec);
+
+  // Key tiles of one KV head are adjacent in launch order (the CTAs of a wave
+  // share a few heads' Q and dO in L2); the low key tiles, which see the most
+  // query tiles under the causal flag, start first.
+  const int bhk = blockIdx.y + blockIdx.z * gridDim.y;  // b * Hkv + hk
+  if (bhk >= p.BHk) return;
+  // A launch whose error word is already set (an earlier wait ran out and
+  // nobody has read the word yet) does no work: its inputs may be invalid.
+  if (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kb = blockIdx.x;                  // key tile
+  const int n0 = kb * kBN;
+  const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
+  const int grp = p.Hq / p.Hkv;
+  const int N = p.N;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&ctl.kv_full, 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&ctl.qdo_full[s], 1);
+      mbar_init(&ctl.qdo_empty[s], 1);
+    }
+    mbar_init(&ctl.sp_full, 1);
+    mbar_init(&ctl.p_ready, 4);
+    mbar_init(&ctl.dq_full, 1);
+    mbar_init(&ctl.dq_free, 4);
+    mbar_init(&ctl.acc_done, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&ctl.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 3) {
+    // Query tiles that can see this key tile, in increasing order.
+    const int nqt = (N + MQ - 1) / MQ;
+    const int qt_lo = p.causal ? n0 / MQ : 0;
+    int count = 0;
+    for (int t0 = qt_lo; t0 < nqt; t0 += 32) {
+      const int qt = t0 + lane;
+      const bool vis = qt < nqt && (!p.mask || p.mask[(size_t)((qt * MQ) / 128) * p.nb + kb]);
+      const unsigned bal = __ballot_sync(0xffffffffu, vis);
+      if (vis) ctl.qtiles[count + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(qt);
+      count += __popc(bal);
+    }
+    if (lane == 0) ctl.nq = count;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = ctl.tmem_base;
+  const int nq = ctl.nq;
+  const int n_items = nq * grp;
+  const Guard g{&ctl.abort, p.err};
+  // item i -> (query head, first query row)
+  auto item_bh = [&](int i) { return b * p.Hq + hk * grp + i / nq; };
+  auto item_q0 = [&](int i) { return static_cast<int>(ctl.qtiles[i % nq]) * MQ; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_items > 0) {
+      prefetch_tmap(&p.tq);
+      prefetch_tmap(&p.tdo);
+      prefetch_tmap(&p.tk);
+      prefetch_tmap(&p.tv);
+      mbar_expect_tx(&ctl.kv_full, 2 * C::kKVBytes);
+      for (int cb = 0; cb < D / 64; ++cb) {
+        tma_load_3d(base + C::kOffK + cb * kBN * 128, &p.tk, &ctl.kv_full, cb * 64, n0, bhk);
+        tma_load_3d(base + C::kOffV + cb * kBN * 128, &p.tv, &ctl.kv_full, cb * 64, n0, bhk);
+      }
+      int issued = 0;
+      for (int i = 0; i < n_items; ++i) {
+        const int s = i % kStages;
+        if (i >= kStages && !mbar_wait(&ctl.qdo_empty[s], ((i / kStages) - 1) & 1, g)) break;
+        const int bh = item_bh(i), q0 = item_q0(i);
+        mbar_expect_tx(&ctl.qdo_full[s], 2 * C::kQBytes + 2 * MQ * 4);
+        for (int cb = 0; cb < D / 64; ++cb) {
+          tma_load_3d(base + C::kOffQ + s * C::kQBytes + cb * C::kQBlock, &p.tq,
+                      &ctl.qdo_full[s], cb * 64, q0, bh);
+          tma_load_3d(base + C::kOffDO + s * C::kQBytes + cb * C::kQBlock, &p.tdo,
+                      &ctl.qdo_full[s], cb * 64, q0, bh);
+        }
+        const size_t vo = (size_t)bh * p.Npad + q0;
+        bulk_load(vec + (s * 2 + 0) * MQ, p.lse2 + vo, MQ * 4, &ctl.qdo_full[s]);
+        bulk_load(vec + (s * 2 + 1) * MQ, p.dvec + vo, MQ * 4, &ctl.qdo_full[s]);
+        issued = i + 1;
+      }
+      drain_wait(&ctl.kv_full, 0);
+      for (int s = 0; s < kStages && s < issued; ++s)
+        drain_wait(&ctl.qdo_full[s], (((issued - 1 - s) / kStages + 1) - 1) & 1);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && n_items > 0) {
+      constexpr uint32_t idSP = idesc_bf16(kBN, MQ, false, false);   // K-major A and B
+      constexpr uint32_t idKV = idesc_bf16(kBN, D, false, true);     // B MN-major
+      constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);      // both MN-major
+      const uint32_t ka = smem_u32(base + C::kOffK), va = smem_u32(base + C::kOffV);
+      const uint32_t qa = smem_u32(base + C::kOffQ), da = smem_u32(base + C::kOffDO);
+      const uint32_t dsa = smem_u32(base + C::kOffDS);
+      auto issue_sp = [&](int s) {
+        const uint32_t qs = qa + s * C::kQBytes, ds_ = da + s * C::kQBytes;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t ok = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
+          const uint32_t oq = (kk >> 2) * C::kQBlock + (kk & 3) * 32;
+          mma_ss(tm + C::kS, sdesc_sw128(ka + ok, 16, 1024), sdesc_sw128(qs + oq, 16, 1024), idSP,
+                 kk > 0);
+          mma_ss(tm + C::kDP, sdesc_sw128(va + ok, 16, 1024), sdesc_sw128(ds_ + oq, 16, 1024),
+                 idSP, kk > 0);
+        }
+      };
+      bool ok = mbar_wait(&ctl.kv_full, 0, g) && mbar_wait(&ctl.qdo_full[0], 0, g);
+      if (ok) {
+        tc_fence_after();
+        issue_sp(0);
+        mma_commit(&ctl.sp_full);
+      }
+      for (int i = 0; ok && i < n_items; ++i) {
+        const int s = i % kStages;
+        const uint32_t qs = qa + s * C::kQBytes, dos = da + s * C::kQBytes;
+        const uint32_t dsb = dsa + (i & 1) * C::kDSBytes;
+        if (!(ok = mbar_wait(&ctl.p_ready, i & 1, g))) break;
+        tc_fence_after();
+        // dV += P^T dO_i
+#pragma unroll
+        for (int kk = 0; kk < MQ / 16; ++kk)
+          mma_ts(tm + C::kDV, tm + C::kS + kk * 8, sdesc_sw128(dos + kk * 2048, C::kQBlock, 1024),
+                 idKV, (i > 0 || kk > 0));
+        if (i + 1 < n_items) {
+          const int s2 = (i + 1) % kStages;
+          if (!(ok = mbar_wait(&ctl.qdo_full[s2], ((i + 1) / kStages) & 1, g))) break;
+          tc_fence_after();
+          issue_sp(s2);
+          mma_commit(&ctl.sp_full);
+        }
+        // dK += dS^T Q_i
+#pragma unroll
+        for (int kk = 0; kk < MQ / 16; ++kk)
+          mma_ss(tm + C::kDK, sdesc_sw128(dsb + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(qs + kk * 2048, C::kQBlock, 1024), idKV, (i > 0 || kk > 0));
+        mma_commit(&ctl.qdo_empty[s]);
+        if (i > 0 && !(ok = mbar_wait(&ctl.dq_free, (i - 1) & 1, g))) break;
+        tc_fence_after();
+        // dQ_i (d = 64: dS K, M = query rows) or dQ_i^T (d = 128: K^T dS^T, M = head dim)
+#pragma unroll
+        for (int kk = 0; kk < kBN / 16; ++kk) {
+          if constexpr (D == 128)
+            mma_ss(tm + C::kDQ, sdesc_sw128(ka + kk * 2048, kBN * 128, 1024),
+                   sdesc_sw128(dsb + kk * 2048, kBN * 128, 1024), idQ, kk > 0);
+          else
+            mma_ss(tm + C::kDQ, sdesc_sw128(dsb + kk * 2048, kBN * 128, 1024),
+                   sdesc_sw128(ka + kk * 2048, kBN * 128, 1024), idQ, kk > 0);
+        }
+        mma_commit(&ctl.dq_full);
+      }
+      mma_commit(&ctl.acc_done);
+      drain_wait(&ctl.acc_done, 0);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------------------------ softmax / dS
+    const int wq = warp & 3;
+    const int r = wq * 32 + lane;                 // key row inside the tile
+    const int kv = n0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const float c = p.c;
+    for (int i = 0; i < n_items; ++i) {
+      const int s = i % kStages;
+      if (!mbar_wait(&ctl.sp_full, i & 1, g)) break;
+      if (!mbar_wait(&ctl.qdo_full[s], (i / kStages) & 1, g)) break;
+      tc_fence_after();
+      const int q0 = item_q0(i);
+      const bool need_mask = kv >= N || (p.causal && q0 < n0 + kBN);
+      const float* lse_s = vec + (s * 2 + 0) * MQ;
+      const float* d_s = vec + (s * 2 + 1) * MQ;
+      uint8_t* dsrow = base + C::kOffDS + (i & 1) * C::kDSBytes + r * 128;
+#pragma unroll 1
+      for (int cc = 0; cc < MQ / 32; ++cc) {
+        uint32_t sv[32], dp[32];
+        tmem_ld32x2(tm + C::kS + lane_off + cc * 32, tm + C::kDP + lane_off + cc * 32, sv, dp);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          const int qa_ = q0 + cc * 32 + e;
+          const float4 l2 = *reinterpret_cast<const float4*>(lse_s + ((cc * 32 + e) & ~3));
+          const float4 dd = *reinterpret_cast<const float4*>(d_s + ((cc * 32 + e) & ~3));
+          const float la = (e & 2) ? l2.z : l2.x, lb = (e & 2) ? l2.w : l2.y;
+          const float da_ = (e & 2) ? dd.z : dd.x, db_ = (e & 2) ? dd.w : dd.y;
+          float p0 = ex2(fmaf(__uint_as_float(sv[e]), c, -la));
+          float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), c, -lb));
+          if (need_mask) {
+            if (kv >= N || (p.causal && qa_ < kv)) p0 = 0.f;
+            if (kv >= N || (p.causal && qa_ + 1 < kv)) p1 = 0.f;
+          }
+          const float g0 = p0 * (__uint_as_float(dp[e]) - da_);
+          const float g1 = p1 * (__uint_as_float(dp[e + 1]) - db_);
+          pk[e >> 1] = pack_bf16(p0, p1);
+          dk[e >> 1] = pack_bf16(g0, g1);
+        }
+        // P^T into the first half of the S columns (already read: chunk cc/2 <= cc)
+        tmem_st16(tm + C::kS + lane_off + cc * 16, pk);
+        // dS^T row into the 128B-swizzled K-major buffer: 16-byte chunks of 8 values
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int qc = cc * 32 + k * 8;               // first query column of the chunk
+          const int blk = qc >> 6, ch = (qc & 63) >> 3;
+          uint4 v = make_uint4(dk[k * 4 + 0], dk[k * 4 + 1], dk[k * 4 + 2], dk[k * 4 + 3]);
+          *reinterpret_cast<uint4*>(dsrow + blk * (kBN * 128) + ((ch ^ (r & 7)) << 4)) = v;
+        }
+      }
+      tmem_st_wait();
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.p_ready);
+    }
+    // ------------------------------------------------------------ dK, dV epilogue
+    if (n_items > 0) {
+      mbar_wait(&ctl.acc_done, 0, g);
+      tc_fence_after();
+    }
+    const bool valid = kv < N;
+    const size_t orow = ((size_t)bhk * N + (valid ? kv : 0)) * D;
+#pragma unroll 1
+    for (int which = 0; which < 2; ++which) {
+      const uint32_t col = which ? C::kDV : C::kDK;
+      const float mul = which ? 1.f : p.scale;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        if (n_items > 0) {
+          tmem_ld32(tm + col + lane_off + cc * 32, v);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) v[e] = 0u;
+        }
+        if (!valid) continue;
+        if (p.grad_bf16) {
+          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(which ? p.dV : p.dK) + orow + cc * 32;
+          uint32_t w[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            w[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            reinterpret_cast<uint4*>(out)[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2],
+                                                          w[4 * e + 3]);
+        } else {
+          float* out = static_cast<float*>(which ? p.dV : p.dK) + orow + cc * 32;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            reinterpret_cast<float4*>(out)[e] =
+                make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
+                            __uint_as_float(v[4 * e + 2]) * mul, __uint_as_float(v[4 * e + 3]) * mul);
+        }
+      }
+    }
+  } else if (warp >= 8) {
+    // ------------------------------------------------------------ dQ drain
+    const int wq = warp & 3;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const bool leader = (warp == 8 && lane == 0);
+    uint8_t* stg = base + C::kOffStg;
+    const float sc = p.scale;
+    // Every drain thread runs all iterations (waits return at once after an
+    // abort), so the named barriers below always see all 128 threads.
+    for (int i = 0; i < n_items; ++i) {
+      mbar_wait(&ctl.dq_full, i & 1, g);
+      tc_fence_after();
+      uint32_t v[64];
+      tmem_ld64(tm + C::kDQ + lane_off, v);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.dq_free);
+      if (leader) bulk_wait_read0();   // the previous reduce has read the staging
+      named_sync(1, 128);
+      if constexpr (D == 128) {
+        // lane = head-dim column d = 32*wq + lane; v[q] for q = 0..63
+        uint8_t* box = stg + wq * C::kStgBox + (lane & 3) * 4;
+        const int ch = lane >> 2;
+#pragma unroll
+        for (int q = 0; q < MQ; ++q)
+          *reinterpret_cast<float*>(box + q * 128 + ((ch ^ (q & 7)) << 4)) =
+              __uint_as_float(v[q]) * sc;
+      } else {
+        // lane = query row q = 32*wq + lane; v[d] for d = 0..63
+        const int q = wq * 32 + lane;
+#pragma unroll
+        for (int bx = 0; bx < 2; ++bx)
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int d0 = bx * 32 + k * 4;
+            *reinterpret_cast<float4*>(stg + bx * C::kStgBox + q * 128 + ((k ^ (q & 7)) << 4)) =
+                make_float4(__uint_as_float(v[d0]) * sc, __uint_as_float(v[d0 + 1]) * sc,
+                            __uint_as_float(v[d0 + 2]) * sc, __uint_as_float(v[d0 + 3]) * sc);
+          }
+      }
+      fence_async_smem();
+      named_sync(1, 128);
+      if (leader) {
+        const int bh = item_bh(i), q0 = item_q0(i);
+#pragma unroll
+        for (int bx = 0; bx < D / 32; ++bx)
+          tma_reduce_add_3d(&p.tdq, stg + bx * C::kStgBox, bx * 32, q0, bh);
+        bulk_commit();
+      }
+    }
+    if (leader) bulk_wait0();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tm, 512);
+  }
+}
+
+template <int D>
+cudaError_t launch(const Problem& pr) {
+  using C = Cfg<D>;
+  BwdParams kp;
+  memset(&kp, 0, sizeof(kp));
+  const uint64_t BHq = (uint64_t)pr.B * pr.Hq, BHk = (uint64_t)pr.B * pr.Hkv;
+  const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_tmap_3d(&kp.tq, pr.Q, bf, 2, D, pr.N, BHq, 64, C::MQ, sw) ||
+      !make_tmap_3d(&kp.tdo, pr.dO, bf, 2, D, pr.N, BHq, 64, C::MQ, sw) ||
+      !make_tmap_3d(&kp.tk, pr.K, bf, 2, D, pr.N, BHk, 64, kBN, sw) ||
+      !make_tmap_3d(&kp.tv, pr.V, bf, 2, D, pr.N, BHk, 64, kBN, sw) ||
+      !make_tmap_3d(&kp.tdq, pr.dQacc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, pr.N, BHq, 32,
+                    C::MQ, sw))
+    return cudaErrorInvalidValue;
+  kp.lse2 = pr.LSE2ws;
+  kp.dvec = pr.Dws;
+  kp.dK = pr.dK;
+  kp.dV = pr.dV;
+  kp.mask = pr.mask;
+  kp.err = pr.err;
+  kp.N = pr.N;
+  kp.Npad = pr.Npad;
+  kp.Hq = pr.Hq;
+  kp.Hkv = pr.Hkv;
+  kp.nb = pr.nb;
+  kp.causal = pr.causal;
+  kp.grad_bf16 = pr.grad_dtype == 1;
+  kp.c = pr.scale * kLog2e;
+  kp.scale = pr.scale;
+  const size_t smem = sizeof(Ctl) + 1024 + C::kOffEnd;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(bwd_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  kp.BHk = (int)BHk;
+  const unsigned ny = (unsigned)std::min<uint64_t>(BHk, 65535);
+  dim3 grid((unsigned)pr.nb, ny, (unsigned)((BHk + ny - 1) / ny));
+  bwd_kernel<D><<<grid, kThreads, smem, pr.stream>>>(kp);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool sm100_bwd_supported(const Problem& p) {
+  const int mq = (p.d == 64) ? 128 : 64;
+  return p.dtype == 1 && (p.d == 64 || p.d == 128) && p.scale > 0.f &&
+         (p.N + mq - 1) / mq <= kMaxQTiles && p.nb <= 65535 && (long long)p.B * p.Hkv <= 65535ll * 65535ll &&
+         (long long)p.B * p.Hkv < (1ll << 31);
+}
+
+// dQ is accumulated in fp32 by TMA reduce-adds: into dQ itself for fp32
+// gradients, into the workspace accumulator (then converted) for bf16.
+bool sm100_bwd_uses_dq_accumulator(const Problem& p) { return p.grad_dtype == 1; }
+
+cudaError_t sm100_bwd_main(const Problem& p) {
+  return p.d == 64 ? launch<64>(p) : launch<128>(p);
+}
+
 }  // namespace fa

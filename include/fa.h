@@ -41,8 +41,10 @@
  * implemented: e.g. fp32 inputs with the tensor-core path). A failed launch
  * returns FA_ERR_CUDA. Every wait inside a kernel is bounded; a wait that runs
  * out sets a bit in the workspace's error word, the kernel returns without
- * faulting, and fa_get_device_error reports FA_ERR_TIMEOUT. The library never
- * traps and never resets the device.
+ * faulting, and fa_get_device_error reports FA_ERR_TIMEOUT. While the word is
+ * set, later tensor-core launches on the same workspace return without work
+ * (their outputs are then undefined) until fa_get_device_error clears it. The
+ * library never traps and never resets the device.
  */
 #ifndef FA_H_
 #define FA_H_
