@@ -7,7 +7,7 @@
 #include <stdint.h>
 #include <stdio.h>
 
-#include "../../include/fa.h"
+#include "fa.h"
 #include "internal.h"
 
 namespace fa {

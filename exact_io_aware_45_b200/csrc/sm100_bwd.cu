@@ -18,11 +18,18 @@
 // accumulator fits the 512 TMEM columns; the dQ product is arranged so its
 // M dimension is 128 either way.
 //
-// MMA issue order per item: dV(i), S(i+1), dP(i+1), dK(i), dQ(i). tcgen05.mma
-// operations from one thread run in order, so the softmax of item i+1 (which
-// waits for S(i+1)/dP(i+1)) knows dV(i) has read P^T(i) from the S columns it
-// overwrites, and that item i-1's dK/dQ have read the dS^T buffer it reuses
-// (double-buffered by item parity).
+// Schedule (d = 128): two sets of S^T / dP^T columns in TMEM alternate
+// between items, so the softmax of item i+1 runs while the tensor core does
+// dV(i), dK(i), dQ(i). MMA issue order for item i: dV(i), dK(i), dQ(i) (into
+// the S columns of its own set, which dV(i) has finished reading: tcgen05.mma
+// operations issued by one thread run in order), then dP(i+2) and, once the
+// drain warps have read dQ(i), S(i+2) into the same set. Q / dO use a
+// three-stage ring.
+// Schedule (d = 64, where two sets do not fit): one set; order dV(i),
+// S(i+1), dP(i+1), dK(i), dQ(i) into its own columns.
+// In both, the dS^T shared buffer alternates by item parity and the softmax
+// of item i only writes it after the MMAs that read it two items earlier
+// have completed (they precede the S MMA it waited for).
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
 // TMEM allocator, warp 3 builds the query-tile list, warps 4-7 softmax / dS
@@ -41,21 +48,26 @@ using namespace sm100;
 constexpr int kBN = 128;            // keys per CTA
 constexpr int kMaxQTiles = 4096;    // query tiles per sequence
 constexpr int kThreads = 384;
-constexpr int kStages = 2;          // Q / dO ring depth
+constexpr int kChunk = 8;           // KV heads interleaved in launch order
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
+  static constexpr bool kDbl = (D == 128);                // two S/dP sets in TMEM
   static constexpr int MQ = (D == 64) ? 128 : 64;         // query rows per item
+  static constexpr int kStages = kDbl ? 3 : 2;            // Q / dO ring depth
   static constexpr int kKVBytes = kBN * D * 2;            // K or V tile
   static constexpr int kQBytes = MQ * D * 2;              // Q or dO tile
   static constexpr int kQBlock = MQ * 128;                // one 64-column block of Q / dO
   static constexpr int kDSBytes = kBN * MQ * 2;           // dS^T buffer (bf16)
-  static constexpr int kStgBytes = MQ * D * 4;            // dQ staging (fp32)
-  static constexpr int kStgBox = MQ * 128;                // one 32-column fp32 box
+  static constexpr int kStgBox = MQ * 128;                // one 32-column fp32 box of dQ
+  static constexpr int kStgBoxes = kDbl ? 2 : D / 32;     // boxes staged at a time
   // TMEM columns
-  static constexpr uint32_t kDK = 0, kDV = D, kS = 2 * D, kDP = 2 * D + MQ,
-                            kDQ = 2 * D + 2 * MQ;
+  static constexpr uint32_t kDK = 0, kDV = D;
+  static constexpr uint32_t kS0 = 2 * D, kDP0 = 2 * D + MQ;
+  static constexpr uint32_t kS1 = kDbl ? 2 * D + 2 * MQ : kS0;
+  static constexpr uint32_t kDP1 = kDbl ? 2 * D + 3 * MQ : kDP0;
+  static constexpr uint32_t kDQ = 2 * D + 2 * MQ;         // dQ columns of the one-set schedule
   // shared memory (offsets from a 1024-aligned base)
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kKVBytes;
@@ -63,15 +75,15 @@ struct Cfg {
   static constexpr int kOffDO = kOffQ + kStages * kQBytes;
   static constexpr int kOffDS = kOffDO + kStages * kQBytes;
   static constexpr int kOffStg = kOffDS + 2 * kDSBytes;
-  static constexpr int kOffVec = kOffStg + kStgBytes;       // [stage][LSE2 | D][MQ] floats
+  static constexpr int kOffVec = kOffStg + kStgBoxes * kStgBox;   // [stage][LSE2 | D][MQ]
   static constexpr int kOffEnd = kOffVec + kStages * 2 * MQ * 4;
-  static_assert(kDQ + 64 <= 512, "TMEM budget");
+  static_assert((kDbl ? kDP1 + MQ : kDQ + 64) <= 512, "TMEM budget");
 };
 
 struct alignas(16) Ctl {
   uint64_t kv_full;
-  uint64_t qdo_full[kStages], qdo_empty[kStages];
-  uint64_t sp_full, p_ready, dq_full, dq_free, acc_done;
+  uint64_t qdo_full[3], qdo_empty[3];
+  uint64_t sp_full[2], p_ready, dq_full, dq_free, acc_done;
   uint32_t tmem_base;
   int abort;
   int nq;                      // visible query tiles per query head
@@ -111,16 +123,15 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   uint8_t* base = smem_raw + (base_addr - raw_addr);
   float* vec = reinterpret_cast<float*>(base + C::kOffVec);
 
-  // Key tiles of one KV head are adjacent in launch order (the CTAs of a wave
-  // share a few heads' Q and dO in L2); the low key tiles, which see the most
-  // query tiles under the causal flag, start first.
-  const int bhk = blockIdx.y + blockIdx.z * gridDim.y;  // b * Hkv + hk
-  if (bhk >= p.BHk) return;
+  // KV heads are taken kChunk at a time (their Q/dO stay in L2 during a
+  // wave); inside a chunk the low key tiles, which see the most query tiles
+  // under the causal flag, start first.
+  int bhk, kb;
+  chunked_order(blockIdx.x, p.nb, p.BHk, kChunk, bhk, kb);
   // A launch whose error word is already set (an earlier wait ran out and
   // nobody has read the word yet) does no work: its inputs may be invalid.
   if (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kb = blockIdx.x;                  // key tile
   const int n0 = kb * kBN;
   const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
   const int grp = p.Hq / p.Hkv;
@@ -128,11 +139,12 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl.kv_full, 1);
-    for (int s = 0; s < kStages; ++s) {
+    for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&ctl.qdo_full[s], 1);
       mbar_init(&ctl.qdo_empty[s], 1);
     }
-    mbar_init(&ctl.sp_full, 1);
+    mbar_init(&ctl.sp_full[0], 1);
+    mbar_init(&ctl.sp_full[1], 1);
     mbar_init(&ctl.p_ready, 4);
     mbar_init(&ctl.dq_full, 1);
     mbar_init(&ctl.dq_free, 4);
@@ -168,6 +180,10 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
   // item i -> (query head, first query row)
   auto item_bh = [&](int i) { return b * p.Hq + hk * grp + i / nq; };
   auto item_q0 = [&](int i) { return static_cast<int>(ctl.qtiles[i % nq]) * MQ; };
+  // TMEM columns of item i
+  auto s_col = [&](int i) { return (i & 1) ? C::kS1 : C::kS0; };
+  auto dp_col = [&](int i) { return (i & 1) ? C::kDP1 : C::kDP0; };
+  auto dq_col = [&](int i) { return C::kDbl ? s_col(i) : C::kDQ; };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -183,8 +199,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       }
       int issued = 0;
       for (int i = 0; i < n_items; ++i) {
-        const int s = i % kStages;
-        if (i >= kStages && !mbar_wait(&ctl.qdo_empty[s], ((i / kStages) - 1) & 1, g)) break;
+        const int s = i % C::kStages;
+        if (i >= C::kStages && !mbar_wait(&ctl.qdo_empty[s], ((i / C::kStages) - 1) & 1, g)) break;
         const int bh = item_bh(i), q0 = item_q0(i);
         mbar_expect_tx(&ctl.qdo_full[s], 2 * C::kQBytes + 2 * MQ * 4);
         for (int cb = 0; cb < D / 64; ++cb) {
@@ -199,8 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
         issued = i + 1;
       }
       drain_wait(&ctl.kv_full, 0);
-      for (int s = 0; s < kStages && s < issued; ++s)
-        drain_wait(&ctl.qdo_full[s], (((issued - 1 - s) / kStages + 1) - 1) & 1);
+      for (int s = 0; s < C::kStages && s < issued; ++s)
+        drain_wait(&ctl.qdo_full[s], (((issued - 1 - s) / C::kStages + 1) - 1) & 1);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -211,61 +227,108 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       const uint32_t ka = smem_u32(base + C::kOffK), va = smem_u32(base + C::kOffV);
       const uint32_t qa = smem_u32(base + C::kOffQ), da = smem_u32(base + C::kOffDO);
       const uint32_t dsa = smem_u32(base + C::kOffDS);
-      auto issue_sp = [&](int s) {
-        const uint32_t qs = qa + s * C::kQBytes, ds_ = da + s * C::kQBytes;
+      auto qstage = [&](int i) { return qa + (i % C::kStages) * C::kQBytes; };
+      auto dostage = [&](int i) { return da + (i % C::kStages) * C::kQBytes; };
+      auto dsbuf = [&](int i) { return dsa + (i & 1) * C::kDSBytes; };
+      auto issue_s = [&](int i) {   // S^T = K Q_i^T
+        const uint32_t qs = qstage(i);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ok = (kk >> 2) * (kBN * 128) + (kk & 3) * 32;
-          const uint32_t oq = (kk >> 2) * C::kQBlock + (kk & 3) * 32;
-          mma_ss(tm + C::kS, sdesc_sw128(ka + ok, 16, 1024), sdesc_sw128(qs + oq, 16, 1024), idSP,
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tm + s_col(i),
+                 sdesc_sw128(ka + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(qs + (kk >> 2) * C::kQBlock + (kk & 3) * 32, 16, 1024), idSP,
                  kk > 0);
-          mma_ss(tm + C::kDP, sdesc_sw128(va + ok, 16, 1024), sdesc_sw128(ds_ + oq, 16, 1024),
-                 idSP, kk > 0);
-        }
       };
-      bool ok = mbar_wait(&ctl.kv_full, 0, g) && mbar_wait(&ctl.qdo_full[0], 0, g);
-      if (ok) {
-        tc_fence_after();
-        issue_sp(0);
-        mma_commit(&ctl.sp_full);
-      }
-      for (int i = 0; ok && i < n_items; ++i) {
-        const int s = i % kStages;
-        const uint32_t qs = qa + s * C::kQBytes, dos = da + s * C::kQBytes;
-        const uint32_t dsb = dsa + (i & 1) * C::kDSBytes;
-        if (!(ok = mbar_wait(&ctl.p_ready, i & 1, g))) break;
-        tc_fence_after();
-        // dV += P^T dO_i
+      auto issue_dp = [&](int i) {  // dP^T = V dO_i^T
+        const uint32_t ds_ = dostage(i);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(tm + dp_col(i),
+                 sdesc_sw128(va + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
+                 sdesc_sw128(ds_ + (kk >> 2) * C::kQBlock + (kk & 3) * 32, 16, 1024), idSP,
+                 kk > 0);
+      };
+      auto issue_dv = [&](int i) {  // dV += P^T dO_i (P^T bf16 in the S columns)
+        const uint32_t dos = dostage(i);
 #pragma unroll
         for (int kk = 0; kk < MQ / 16; ++kk)
-          mma_ts(tm + C::kDV, tm + C::kS + kk * 8, sdesc_sw128(dos + kk * 2048, C::kQBlock, 1024),
-                 idKV, (i > 0 || kk > 0));
-        if (i + 1 < n_items) {
-          const int s2 = (i + 1) % kStages;
-          if (!(ok = mbar_wait(&ctl.qdo_full[s2], ((i + 1) / kStages) & 1, g))) break;
-          tc_fence_after();
-          issue_sp(s2);
-          mma_commit(&ctl.sp_full);
-        }
-        // dK += dS^T Q_i
+          mma_ts(tm + C::kDV, tm + s_col(i) + kk * 8,
+                 sdesc_sw128(dos + kk * 2048, C::kQBlock, 1024), idKV, (i > 0 || kk > 0));
+      };
+      auto issue_dk = [&](int i) {  // dK += dS^T Q_i
+        const uint32_t qs = qstage(i), dsb = dsbuf(i);
 #pragma unroll
         for (int kk = 0; kk < MQ / 16; ++kk)
-          mma_ss(tm + C::kDK, sdesc_sw128(dsb + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
+          mma_ss(tm + C::kDK,
+                 sdesc_sw128(dsb + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
                  sdesc_sw128(qs + kk * 2048, C::kQBlock, 1024), idKV, (i > 0 || kk > 0));
-        mma_commit(&ctl.qdo_empty[s]);
-        if (i > 0 && !(ok = mbar_wait(&ctl.dq_free, (i - 1) & 1, g))) break;
-        tc_fence_after();
-        // dQ_i (d = 64: dS K, M = query rows) or dQ_i^T (d = 128: K^T dS^T, M = head dim)
+      };
+      auto issue_dq = [&](int i) {  // dQ_i^T = K^T dS_i^T (d = 128) or dQ_i = dS_i K (d = 64)
+        const uint32_t dsb = dsbuf(i);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           if constexpr (D == 128)
-            mma_ss(tm + C::kDQ, sdesc_sw128(ka + kk * 2048, kBN * 128, 1024),
+            mma_ss(tm + dq_col(i), sdesc_sw128(ka + kk * 2048, kBN * 128, 1024),
                    sdesc_sw128(dsb + kk * 2048, kBN * 128, 1024), idQ, kk > 0);
           else
-            mma_ss(tm + C::kDQ, sdesc_sw128(dsb + kk * 2048, kBN * 128, 1024),
+            mma_ss(tm + dq_col(i), sdesc_sw128(dsb + kk * 2048, kBN * 128, 1024),
                    sdesc_sw128(ka + kk * 2048, kBN * 128, 1024), idQ, kk > 0);
         }
-        mma_commit(&ctl.dq_full);
+      };
+      auto wait_q = [&](int i) {
+        return mbar_wait(&ctl.qdo_full[i % C::kStages], (i / C::kStages) & 1, g);
+      };
+      bool ok = mbar_wait(&ctl.kv_full, 0, g) && wait_q(0);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+        issue_dp(0);
+        mma_commit(&ctl.sp_full[0]);
+      }
+      if constexpr (C::kDbl) {
+        if (ok && n_items > 1 && (ok = wait_q(1))) {
+          tc_fence_after();
+          issue_s(1);
+          issue_dp(1);
+          mma_commit(&ctl.sp_full[1]);
+        }
+        for (int i = 0; ok && i < n_items; ++i) {
+          if (!(ok = mbar_wait(&ctl.p_ready, i & 1, g))) break;
+          tc_fence_after();
+          issue_dv(i);
+          issue_dk(i);
+          mma_commit(&ctl.qdo_empty[i % C::kStages]);
+          issue_dq(i);
+          mma_commit(&ctl.dq_full);
+          if (i + 2 < n_items) {
+            if (!(ok = wait_q(i + 2))) break;
+            tc_fence_after();
+            issue_dp(i + 2);
+            if (!(ok = mbar_wait(&ctl.dq_free, i & 1, g))) break;   // dQ(i) drained
+            tc_fence_after();
+            issue_s(i + 2);
+            mma_commit(&ctl.sp_full[i & 1]);
+          }
+        }
+      } else {
+        for (int i = 0; ok && i < n_items; ++i) {
+          if (!(ok = mbar_wait(&ctl.p_ready, i & 1, g))) break;
+          tc_fence_after();
+          issue_dv(i);
+          if (i + 1 < n_items) {
+            if (!(ok = wait_q(i + 1))) break;
+            tc_fence_after();
+            issue_s(i + 1);
+            issue_dp(i + 1);
+            mma_commit(&ctl.sp_full[0]);
+          }
+          issue_dk(i);
+          mma_commit(&ctl.qdo_empty[i % C::kStages]);
+          if (i > 0 && !(ok = mbar_wait(&ctl.dq_free, (i - 1) & 1, g))) break;
+          tc_fence_after();
+          issue_dq(i);
+          mma_commit(&ctl.dq_full);
+        }
       }
       mma_commit(&ctl.acc_done);
       drain_wait(&ctl.acc_done, 0);
@@ -278,9 +341,11 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float c = p.c;
     for (int i = 0; i < n_items; ++i) {
-      const int s = i % kStages;
-      if (!mbar_wait(&ctl.sp_full, i & 1, g)) break;
-      if (!mbar_wait(&ctl.qdo_full[s], (i / kStages) & 1, g)) break;
+      const int s = i % C::kStages;
+      const bool spok = C::kDbl ? mbar_wait(&ctl.sp_full[i & 1], (i >> 1) & 1, g)
+                                : mbar_wait(&ctl.sp_full[0], i & 1, g);
+      if (!spok) break;
+      if (!mbar_wait(&ctl.qdo_full[s], (i / C::kStages) & 1, g)) break;
       tc_fence_after();
       const int q0 = item_q0(i);
       const bool need_mask = kv >= N || (p.causal && q0 < n0 + kBN);
@@ -290,7 +355,8 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
 #pragma unroll 1
       for (int cc = 0; cc < MQ / 32; ++cc) {
         uint32_t sv[32], dp[32];
-        tmem_ld32x2(tm + C::kS + lane_off + cc * 32, tm + C::kDP + lane_off + cc * 32, sv, dp);
+        tmem_ld32x2(tm + s_col(i) + lane_off + cc * 32, tm + dp_col(i) + lane_off + cc * 32, sv,
+                    dp);
         uint32_t pk[16], dk[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
@@ -311,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
           dk[e >> 1] = pack_bf16(g0, g1);
         }
         // P^T into the first half of the S columns (already read: chunk cc/2 <= cc)
-        tmem_st16(tm + C::kS + lane_off + cc * 16, pk);
+        tmem_st16(tm + s_col(i) + lane_off + cc * 16, pk);
         // dS^T row into the 128B-swizzled K-major buffer: 16-byte chunks of 8 values
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
@@ -381,22 +447,38 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
       mbar_wait(&ctl.dq_full, i & 1, g);
       tc_fence_after();
       uint32_t v[64];
-      tmem_ld64(tm + C::kDQ + lane_off, v);
+      tmem_ld64(tm + dq_col(i) + lane_off, v);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.dq_free);
-      if (leader) bulk_wait_read0();   // the previous reduce has read the staging
-      named_sync(1, 128);
+      const int bh = item_bh(i), q0 = item_q0(i);
       if constexpr (D == 128) {
-        // lane = head-dim column d = 32*wq + lane; v[q] for q = 0..63
-        uint8_t* box = stg + wq * C::kStgBox + (lane & 3) * 4;
+        // lane = head-dim column d = 32*wq + lane; v[q] for q = 0..63. Two
+        // 16 KB halves: warps 0-1 stage d 0..63, then warps 2-3 stage 64..127.
+        uint8_t* box = stg + (wq & 1) * C::kStgBox + (lane & 3) * 4;
         const int ch = lane >> 2;
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+          if (leader) bulk_wait_read0();   // the previous reduce has read the staging
+          named_sync(1, 128);
+          if ((wq >> 1) == hf) {
 #pragma unroll
-        for (int q = 0; q < MQ; ++q)
-          *reinterpret_cast<float*>(box + q * 128 + ((ch ^ (q & 7)) << 4)) =
-              __uint_as_float(v[q]) * sc;
+            for (int q = 0; q < MQ; ++q)
+              *reinterpret_cast<float*>(box + q * 128 + ((ch ^ (q & 7)) << 4)) =
+                  __uint_as_float(v[q]) * sc;
+            fence_async_smem();
+          }
+          named_sync(1, 128);
+          if (leader) {
+            tma_reduce_add_3d(&p.tdq, stg, (2 * hf) * 32, q0, bh);
+            tma_reduce_add_3d(&p.tdq, stg + C::kStgBox, (2 * hf + 1) * 32, q0, bh);
+            bulk_commit();
+          }
+        }
       } else {
         // lane = query row q = 32*wq + lane; v[d] for d = 0..63
+        if (leader) bulk_wait_read0();
+        named_sync(1, 128);
         const int q = wq * 32 + lane;
 #pragma unroll
         for (int bx = 0; bx < 2; ++bx)
@@ -407,15 +489,14 @@ __global__ void __launch_bounds__(kThreads, 1) bwd_kernel(const __grid_constant_
                 make_float4(__uint_as_float(v[d0]) * sc, __uint_as_float(v[d0 + 1]) * sc,
                             __uint_as_float(v[d0 + 2]) * sc, __uint_as_float(v[d0 + 3]) * sc);
           }
-      }
-      fence_async_smem();
-      named_sync(1, 128);
-      if (leader) {
-        const int bh = item_bh(i), q0 = item_q0(i);
+        fence_async_smem();
+        named_sync(1, 128);
+        if (leader) {
 #pragma unroll
-        for (int bx = 0; bx < D / 32; ++bx)
-          tma_reduce_add_3d(&p.tdq, stg + bx * C::kStgBox, bx * 32, q0, bh);
-        bulk_commit();
+          for (int bx = 0; bx < D / 32; ++bx)
+            tma_reduce_add_3d(&p.tdq, stg + bx * C::kStgBox, bx * 32, q0, bh);
+          bulk_commit();
+        }
       }
     }
     if (leader) bulk_wait0();
@@ -468,8 +549,7 @@ cudaError_t launch(const Problem& pr) {
     attr_set = true;
   }
   kp.BHk = (int)BHk;
-  const unsigned ny = (unsigned)std::min<uint64_t>(BHk, 65535);
-  dim3 grid((unsigned)pr.nb, ny, (unsigned)((BHk + ny - 1) / ny));
+  dim3 grid((unsigned)(BHk * pr.nb));
   bwd_kernel<D><<<grid, kThreads, smem, pr.stream>>>(kp);
   count_launch();
   return cudaGetLastError();
@@ -480,7 +560,7 @@ cudaError_t launch(const Problem& pr) {
 bool sm100_bwd_supported(const Problem& p) {
   const int mq = (p.d == 64) ? 128 : 64;
   return p.dtype == 1 && (p.d == 64 || p.d == 128) && p.scale > 0.f &&
-         (p.N + mq - 1) / mq <= kMaxQTiles && p.nb <= 65535 && (long long)p.B * p.Hkv <= 65535ll * 65535ll &&
+         (p.N + mq - 1) / mq <= kMaxQTiles && (long long)p.B * p.Hkv * p.nb < (1ll << 31) &&
          (long long)p.B * p.Hkv < (1ll << 31);
 }
 

@@ -135,6 +135,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Maps a linear CTA index to (head, block) so that the blocks of `chunk`
+// heads are interleaved and, inside the chunk, issued from block 0 to
+// block nblk-1 (callers order their blocks by decreasing work). A wave then
+// covers only a few heads (their K/V or Q/dO stay in L2) while the longest
+// blocks of each chunk start first.
+__device__ __forceinline__ void chunked_order(int lin, int nblk, int BH, int chunk, int& head,
+                                              int& blk) {
+  const int per = chunk * nblk;
+  const int c = lin / per, rem = lin - c * per;
+  const int heads = min(chunk, BH - c * chunk);
+  blk = rem / heads;
+  head = c * chunk + (rem - blk * heads);
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m) {

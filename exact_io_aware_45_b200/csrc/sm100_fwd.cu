@@ -33,6 +33,8 @@
 // tile 0, warps 8-11 softmax of query tile 1.
 #include <math.h>
 
+#include <algorithm>
+
 #include "sm100_common.cuh"
 
 namespace fa {
@@ -46,6 +48,7 @@ constexpr int kThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kTau = 8.0f;       // reference-max slack, log2 units
+constexpr int kChunk = 16;         // heads interleaved in launch order
 
 template <int D>
 struct Cfg {
@@ -81,7 +84,7 @@ struct FwdParams {
   float* LSE;
   const uint8_t* mask;
   unsigned* err;
-  int N, Hq, Hkv, nb, nblk, causal;
+  int N, Hq, Hkv, nb, nblk, causal, BH;
   float c;                   // scale * log2(e)
 };
 
@@ -102,9 +105,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   const uint32_t tile_addr = (raw_addr + sizeof(Ctl) + 1023u) & ~1023u;
   uint8_t* tiles_base = smem_raw + (tile_addr - raw_addr);
 
+  // Heads are taken kChunk at a time (their K/V stay in L2 during a wave);
+  // inside a chunk the query blocks with the longest causal rows start first.
+  int bh, rblk;
+  chunked_order(blockIdx.x, p.nblk, p.BH, kChunk, bh, rblk);
+  // A launch whose error word is already set (an earlier wait ran out and
+  // nobody has read the word yet) does no work: its inputs may be invalid.
+  if (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bh = blockIdx.x;                     // b * Hq + h
-  const int blk = p.nblk - 1 - blockIdx.y;       // longest causal rows first
+  const int blk = p.nblk - 1 - rblk;
   const int h = bh % p.Hq, b = bh / p.Hq;
   const int bhk = b * p.Hkv + h / (p.Hq / p.Hkv);
   const int q0 = blk * 2 * kBM;
@@ -271,25 +280,30 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       if (!mbar_wait(&ctl.s_full[t], j & 1, g)) break;
       tc_fence_after();
       uint32_t sr[128];
-      tmem_ld64(sreg, *reinterpret_cast<uint32_t(*)[64]>(&sr[0]));
-      tmem_ld64(sreg + 64, *reinterpret_cast<uint32_t(*)[64]>(&sr[64]));
+      tmem_ld128(sreg, sr);
       const int col0 = ctl.tiles[j] * kBN;
       const bool dead = (ctl.dead[j] >> t) & 1;
       const bool need_mask = dead || col0 + kBN > N || (p.causal && col0 + kBN - 1 > tile_row0);
-      float mx = -INFINITY;
       if (need_mask) {
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
           const int col = col0 + i;
           const bool bad = dead || col >= N || (p.causal && col > row);
-          const float v = bad ? -INFINITY : __uint_as_float(sr[i]);
-          sr[i] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          if (bad) sr[i] = __float_as_uint(-INFINITY);
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 128; ++i) mx = fmaxf(mx, __uint_as_float(sr[i]));
       }
+      // Row maximum: eight independent chains of three-input max.
+      float m8[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const float* v = reinterpret_cast<const float*>(&sr[16 * k]);
+        float m = fmax3(v[0], v[1], v[2]);
+#pragma unroll
+        for (int i = 3; i < 15; i += 2) m = fmax3(m, v[i], v[i + 1]);
+        m8[k] = fmaxf(m, v[15]);
+      }
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                             fmaxf(m8[6], m8[7]));
       const float mx2 = mx * c;
       const bool grow = mx2 > m_ref + kTau;
       float alpha = 1.f;
@@ -299,17 +313,27 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         l *= alpha;
       }
       const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-      uint32_t pk[64];
-      float sum0 = 0.f, sum1 = 0.f;
+      // p = 2^(s*c - mu), two lanes per FMA, four pair accumulators for the
+      // sum; P goes to TMEM half a row at a time to keep registers free.
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
+      const float2 c2 = make_float2(c, c), nmu2 = make_float2(-mu, -mu);
 #pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const float p0 = ex2(fmaf(__uint_as_float(sr[2 * i]), c, -mu));
-        const float p1 = ex2(fmaf(__uint_as_float(sr[2 * i + 1]), c, -mu));
-        sum0 += p0;
-        sum1 += p1;
-        pk[i] = pack_bf16(p0, p1);
+      for (int hf = 0; hf < 2; ++hf) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int k = 64 * hf + 2 * i;
+          const float2 x =
+              ffma2(make_float2(__uint_as_float(sr[k]), __uint_as_float(sr[k + 1])), c2, nmu2);
+          const float2 e = make_float2(ex2(x.x), ex2(x.y));
+          acc[i & 3] = fadd2(acc[i & 3], e);
+          pk[i] = pack_bf16(e.x, e.y);
+        }
+        tmem_st32(sreg + C::kPOff + 32 * hf, pk);
       }
-      l += sum0 + sum1;
+      const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+      l += (a01.x + a01.y) + (a23.x + a23.y);
       // The accumulator holds P V of earlier tiles (complete: the commit that
       // signalled S_t came after them); rescale it where the reference moved.
       if (__any_sync(0xffffffffu, grow && j > 0)) {
@@ -322,8 +346,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           tmem_st32(oreg + cc * 32, o);
         }
       }
-      tmem_st32(sreg + C::kPOff, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-      tmem_st32(sreg + C::kPOff + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
@@ -399,7 +421,8 @@ cudaError_t launch(const Problem& pr) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  dim3 grid((unsigned)BHq, (unsigned)kp.nblk);
+  kp.BH = (int)BHq;
+  dim3 grid((unsigned)(BHq * kp.nblk));
   fwd_kernel<D><<<grid, kThreads, smem, pr.stream>>>(kp);
   count_launch();
   return cudaGetLastError();
@@ -409,7 +432,7 @@ cudaError_t launch(const Problem& pr) {
 
 bool sm100_fwd_supported(const Problem& p) {
   return p.dtype == 1 && (p.d == 64 || p.d == 128) && p.scale > 0.f && p.nb <= kMaxTiles &&
-         (long long)p.B * p.Hq < (1ll << 31);
+         (long long)p.B * p.Hq * ((p.N + 255) / 256) < (1ll << 31);
 }
 
 cudaError_t sm100_fwd(const Problem& p) {

@@ -15,7 +15,9 @@ import os
 from typing import Optional
 
 PKG = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG, "_lib", "libfa.so")
+# FA_LIBRARY may name another build of libfa.so (e.g. one compiled with
+# different tile parameters); the default is the in-tree build.
+LIB_PATH = os.environ.get("FA_LIBRARY") or os.path.join(PKG, "_lib", "libfa.so")
 
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 FA_F32, FA_BF16 = 0, 1
