@@ -11,7 +11,7 @@ rounding of the bf16 P it feeds.
 
 prints the four coefficients (c0 + c1 f + c2 f^2 + c3 f^3) as float32 and
 the maximum relative error of the float32 evaluation, the numbers the kernel
-source carries.
+source carries (kExp2P0..kExp2P3 in sm100_common.cuh).
 """
 import numpy as np
 
@@ -26,9 +26,9 @@ def fit(degree: int = 3, nodes: int = 4096):
 
 
 def eval_f32(x, c):
-    """The kernel's steps in float32: round x to j with the 1.5*2^23 shift,
+    """The kernel's steps in float32: clamp x at -125, round x to j with the 1.5*2^23 shift,
     f = x - j, Horner cubic, then add j to the exponent field."""
-    x = np.maximum(np.asarray(x, dtype=np.float32), np.float32(-126.0))
+    x = np.maximum(np.asarray(x, dtype=np.float32), np.float32(-125.0))
     magic = np.float32(12582912.0)
     t = (x + magic).astype(np.float32)
     j = (t - magic).astype(np.float32)

@@ -80,6 +80,13 @@ int fa_version(void) { return 10000; }
 
 int fa_last_launch_count(void) { return t_launches; }
 
+fa_status fa_exp2_fma(const float* x, float* y, long long n, void* stream) {
+  t_launches = 0;
+  if (n < 0 || (n > 0 && (!x || !y))) return FA_ERR_INVALID_ARG;
+  if (n > (1ll << 40)) return FA_ERR_UNSUPPORTED;
+  return from_cuda(exp2_fma_eval(x, y, n, static_cast<cudaStream_t>(stream)));
+}
+
 size_t fa_fwd_workspace_size(void) { return kErrBlock; }
 
 size_t fa_bwd_workspace_size(int B, int Hq, int N, int d) {

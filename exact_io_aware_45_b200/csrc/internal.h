@@ -53,6 +53,8 @@ cudaError_t dq_convert(const Problem& p);
 // tcgen05 / TMA kernels for sm_100a. sm100_fwd.cu, sm100_bwd.cu
 bool sm100_fwd_supported(const Problem& p);
 cudaError_t sm100_fwd(const Problem& p);
+// Evaluates the forward kernel's FMA-pipe exp2 on n floats (diagnostic).
+cudaError_t exp2_fma_eval(const float* x, float* y, long long n, cudaStream_t stream);
 bool sm100_bwd_supported(const Problem& p);
 bool sm100_bwd_uses_dq_accumulator(const Problem& p);
 cudaError_t sm100_bwd_main(const Problem& p);

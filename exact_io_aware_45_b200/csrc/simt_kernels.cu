@@ -133,31 +133,45 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(Problem p) {
 
 // D_i = sum_k dO_ik O_ik and LSE2_i = LSE_i * log2(e) (+inf for rows with no
 // visible key and for padding rows), one warp per row of the padded layout.
-template <typename T>
+// D_i = sum_k dO_ik O_ik and LSE_i * log2(e) for every row of the padded
+// [B*Hq][Npad] workspace vectors (padding rows: D = 0, LSE2 = +inf, so their
+// P is 0), optionally zeroing the row of the fp32 dQ accumulator. TPR
+// threads share a row, each reading 16 bytes of O and of dO (VEC elements),
+// and the partial dots are summed with shuffles inside the TPR-lane group.
+template <typename T, int TPR>
 __global__ void __launch_bounds__(256) preprocess_kernel(Problem p, int zero_acc) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int total = p.B * p.Hq * p.Npad;
-  if (warp >= total) return;
-  const int bh = warp / p.Npad, row = warp % p.Npad;
+  constexpr int VEC = 16 / sizeof(T);
+  const long long gt = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long total = (long long)p.B * p.Hq * p.Npad;
+  const long long rowid = gt / TPR;
+  const int part = (int)(gt % TPR);
+  const bool live = rowid < total;   // whole TPR groups are live or not
+  const int bh = live ? (int)(rowid / p.Npad) : 0;
+  const int row = live ? (int)(rowid % p.Npad) : p.N;
   const int d = p.d;
   float acc = 0.f;
-  float lse2 = INFINITY;
-  if (row < p.N) {
-    const size_t base = ((size_t)bh * p.N + row) * d;
-    const T* o = static_cast<const T*>(p.O) + base;
-    const T* g = static_cast<const T*>(p.dO) + base;
-    for (int k = lane; k < d; k += 32) acc = fmaf(ld<T>(o + k), ld<T>(g + k), acc);
-    const float L = p.LSE[(size_t)bh * p.N + row];
-    if (L != -INFINITY) lse2 = L * kLog2e;
+  if (live && row < p.N) {
+    const size_t off = ((size_t)bh * p.N + row) * d + (size_t)part * VEC;
+    const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.O) + off);
+    const uint4 gv = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.dO) + off);
+    const T* o = reinterpret_cast<const T*>(&ov);
+    const T* g = reinterpret_cast<const T*>(&gv);
+#pragma unroll
+    for (int k = 0; k < VEC; ++k) acc = fmaf(ld<T>(o + k), ld<T>(g + k), acc);
     if (zero_acc) {
-      float* a = p.dQacc + base;
-      for (int k = lane; k < d; k += 32) a[k] = 0.f;
+      float4* a = reinterpret_cast<float4*>(p.dQacc + off);
+#pragma unroll
+      for (int k = 0; k < VEC / 4; ++k) a[k] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
+  for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (live && part == 0) {
+    float lse2 = INFINITY;
+    if (row < p.N) {
+      const float L = p.LSE[(size_t)bh * p.N + row];
+      if (L != -INFINITY) lse2 = L * kLog2e;
+    }
     p.Dws[(size_t)bh * p.Npad + row] = acc;
     p.LSE2ws[(size_t)bh * p.Npad + row] = lse2;
   }
@@ -359,15 +373,30 @@ cudaError_t simt_fwd(const Problem& p) {
   }
 }
 
-cudaError_t bwd_preprocess(const Problem& p, bool zero_acc) {
-  const long long rows = (long long)p.B * p.Hq * p.Npad;
-  const int blocks = (int)((rows + 7) / 8);
-  if (p.dtype == 0)
-    preprocess_kernel<float><<<blocks, 256, 0, p.stream>>>(p, zero_acc ? 1 : 0);
-  else
-    preprocess_kernel<__nv_bfloat16><<<blocks, 256, 0, p.stream>>>(p, zero_acc ? 1 : 0);
+template <typename T, int TPR>
+cudaError_t launch_preprocess(const Problem& p, bool zero_acc) {
+  const long long threads = (long long)p.B * p.Hq * p.Npad * TPR;
+  const long long blocks = (threads + 255) / 256;
+  preprocess_kernel<T, TPR><<<(unsigned)blocks, 256, 0, p.stream>>>(p, zero_acc ? 1 : 0);
   count_launch();
   return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t preprocess_d(const Problem& p, bool zero_acc) {
+  constexpr int VEC = 16 / sizeof(T);
+  switch (p.d / VEC) {
+    case 2: return launch_preprocess<T, 2>(p, zero_acc);
+    case 4: return launch_preprocess<T, 4>(p, zero_acc);
+    case 8: return launch_preprocess<T, 8>(p, zero_acc);
+    case 16: return launch_preprocess<T, 16>(p, zero_acc);
+    case 32: return launch_preprocess<T, 32>(p, zero_acc);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t bwd_preprocess(const Problem& p, bool zero_acc) {
+  return p.dtype == 0 ? preprocess_d<float>(p, zero_acc) : preprocess_d<__nv_bfloat16>(p, zero_acc);
 }
 
 cudaError_t simt_bwd_main(const Problem& p) {

@@ -28,7 +28,7 @@ __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31) == 0; 
 
 __device__ __forceinline__ float ex2(float x) {
   float y;
-  asm volatile("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
@@ -45,24 +45,33 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return r;
 }
 
-// Two-lane fp32 FMA / add on a register pair: (a.x*b.x + c.x, a.y*b.y + c.y).
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 r;
-  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
-      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(r.x), "=f"(r.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return r;
-}
-__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
-  float2 r;
-  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
-      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
-      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
-      : "=f"(r.x), "=f"(r.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
-  return r;
+// Two-lane fp32 FMA / add / multiply (fma.rn.f32x2 and friends).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+
+// 2^x for two lanes on the FMA pipe instead of the MUFU unit. Cody and
+// Waite's range reduction in base 2 splits x = j + f with j = rint(x) and
+// |f| <= 1/2 (adding 1.5 * 2^23 leaves rint(x) in the low mantissa bits of
+// the sum); 2^f is a cubic whose coefficients are the relative-error
+// least-squares fit printed by exp2_poly_fit.py (max relative error 7.7e-5),
+// and 2^j is added to the exponent field. Inputs below -125 are clamped to
+// -125 so the exponent stays normal: the result is then 2^-125 instead of a
+// smaller number. Not for -inf (masked scores): callers use ex2() there.
+constexpr float kExp2P0 = 9.999289513e-01f, kExp2P1 = 6.932762265e-01f,
+                kExp2P2 = 2.426040471e-01f, kExp2P3 = 5.508868396e-02f;
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(kRound, kRound));
+  const float2 j = fadd2(t, make_float2(-kRound, -kRound));
+  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), x);
+  float2 q = ffma2(make_float2(kExp2P3, kExp2P3), f, make_float2(kExp2P2, kExp2P2));
+  q = ffma2(q, f, make_float2(kExp2P1, kExp2P1));
+  q = ffma2(q, f, make_float2(kExp2P0, kExp2P0));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 // Named barrier among `count` threads (a multiple of 32).
@@ -333,6 +342,30 @@ __device__ __forceinline__ void tmem_ld32x2(uint32_t ta, uint32_t tb, uint32_t (
       : "memory");
 #undef FA_Q8
 }
+
+// 32 consecutive columns, asynchronous: the registers are valid only after
+// tmem_wait_ld(r) on the same array (which also orders their later uses).
+__device__ __forceinline__ void tmem_ld32_async(uint32_t ta, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24)
+      : "r"(ta)
+      : "memory");
+}
+
+#define FA_RW8(i) "+r"(r[i + 0]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), \
+                  "+r"(r[i + 4]), "+r"(r[i + 5]), "+r"(r[i + 6]), "+r"(r[i + 7])
+// Waits for this thread's outstanding TMEM loads; `r` is passed through so the
+// compiler cannot move uses of the loaded registers above the wait.
+__device__ __forceinline__ void tmem_wait_ld(uint32_t (&r)[32]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;"
+               : FA_RW8(0), FA_RW8(8), FA_RW8(16), FA_RW8(24)
+               :
+               : "memory");
+}
+#undef FA_RW8
 
 __device__ __forceinline__ void tmem_st_wait() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");

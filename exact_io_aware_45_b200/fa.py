@@ -26,7 +26,7 @@ PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
 # every symbol include/fa.h declares
 EXPORTS = ("fa_status_string", "fa_version", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
            "fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_preprocess", "fa_bwd_main",
-           "fa_bwd_finalize", "fa_last_launch_count", "fa_get_device_error")
+           "fa_bwd_finalize", "fa_last_launch_count", "fa_get_device_error", "fa_exp2_fma")
 
 _lib = None
 
@@ -69,6 +69,8 @@ def lib() -> ctypes.CDLL:
             getattr(L, n).restype = _I
         L.fa_last_launch_count.restype = _I
         L.fa_get_device_error.argtypes = [_P, _P]
+        L.fa_exp2_fma.argtypes = [_P, _P, ctypes.c_longlong, _P]
+        L.fa_exp2_fma.restype = _I
         _lib = L
     return _lib
 
@@ -125,6 +127,10 @@ def fa_last_launch_count() -> int:
 
 def fa_get_device_error(workspace_ptr: int, stream_ptr: int) -> int:
     return lib().fa_get_device_error(workspace_ptr, stream_ptr)
+
+
+def fa_exp2_fma(x_ptr: int, y_ptr: int, n: int, stream_ptr: int) -> int:
+    return lib().fa_exp2_fma(x_ptr, y_ptr, n, stream_ptr)
 
 
 # ------------------------------------------------------------------ torch helpers

@@ -191,6 +191,20 @@ fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void
                          const uint8_t* block_mask, int dtype, unsigned* device_error,
                          void* stream);
 
+/*
+ * Diagnostic: y[i] = 2^x[i] evaluated with the FMA-pipe exponential that the
+ * forward kernel uses for part of its softmax terms (range reduction
+ * x = rint(x) + f, |f| <= 1/2, then a fitted cubic for 2^f; relative error
+ * below 1e-4 for x in [-125, 64]; inputs below -125 give 2^-125). No
+ * passage of the FlashAttention pages defines it: the lesson's Researcher
+ * section ("Version lineage") names software exponentials on Blackwell, and
+ * this entry point lets tests check the one used here against its bound.
+ * x and y are device float arrays of n >= 0 elements (NULL allowed when
+ * n == 0); asynchronous on `stream`. FA_ERR_INVALID_ARG for n < 0 or NULL
+ * pointers with n > 0.
+ */
+fa_status fa_exp2_fma(const float* x, float* y, long long n, void* stream);
+
 /* Number of kernel launches the last successful call of fa_fwd_ex / fa_bwd_ex
  * or one of the stages made from the calling thread (for launch accounting). */
 int fa_last_launch_count(void);
