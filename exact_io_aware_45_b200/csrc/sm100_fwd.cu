@@ -24,7 +24,10 @@
 //
 // Two query tiles alternate on the tensor core (ping-pong): while one
 // softmax warpgroup works on S_0, the MMA warp runs P_1 V and Q_1 K^T, and the
-// other way round. P_t is written into the upper half of S_t's TMEM columns;
+// other way round. Each softmax signals twice per tile: once P of the first
+// 64 keys is in TMEM (the MMA warp starts P V on those keys) and once all of
+// P is; a rescale of O, when the reference max moved, happens before the
+// first signal. P_t is written into the upper half of S_t's TMEM columns;
 // tcgen05.mma operations issued by one thread execute in order, so the next
 // Q_t K^T that overwrites S_t cannot overtake the P_t V that reads it.
 //
@@ -74,7 +77,7 @@ struct Cfg {
 struct alignas(16) Ctl {
   uint64_t q_full;
   uint64_t k_full[4], v_full[4], kv_empty[4];
-  uint64_t s_full[2], p_full[2];
+  uint64_t s_full[2], p_half[2], p_full[2];
   uint64_t o_done;
   uint32_t tmem_base;
   int abort;
@@ -154,6 +157,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&ctl.s_full[t], 1);
+      mbar_init(&ctl.p_half[t], 4);
       mbar_init(&ctl.p_full[t], 4);
     }
     mbar_init(&ctl.o_done, 1);
@@ -246,13 +250,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                  sdesc_sw128(kt + off, 16, 1024), idS, kk > 0);
         }
       };
-      auto issue_pv = [&](int t, int stage, bool acc) {
+      // P V over keys 64*hf .. 64*hf+63 of the tile.
+      auto issue_pv = [&](int t, int stage, bool acc, int hf) {
         const uint32_t vt = va + stage * C::kTileBytes;
         const uint32_t pt = tm + (t ? C::kS1 : C::kS0) + C::kPOff;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk)
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * hf + k4;
           mma_ts(tm + (t ? C::kO1 : C::kO0), pt + kk * 8,
                  sdesc_sw128(vt + kk * 16 * 128, C::kBlockBytes, 1024), idO, (acc || kk > 0));
+        }
       };
       bool ok = mbar_wait(&ctl.q_full, 0, g) && mbar_wait(&ctl.k_full[0], 0, g);
       if (ok) {
@@ -265,10 +272,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       for (int j = 0; ok && j < T; ++j) {
         const int s = j % C::kStages;
         const uint32_t ph = (j / C::kStages) & 1;
-        if (!(ok = mbar_wait(&ctl.v_full[s], ph, g) && mbar_wait(&ctl.p_full[0], j & 1, g)))
+        if (!(ok = mbar_wait(&ctl.v_full[s], ph, g) && mbar_wait(&ctl.p_half[0], j & 1, g)))
           break;
         tc_fence_after();
-        issue_pv(0, s, j > 0);
+        issue_pv(0, s, j > 0, 0);
+        if (!(ok = mbar_wait(&ctl.p_full[0], j & 1, g))) break;
+        tc_fence_after();
+        issue_pv(0, s, j > 0, 1);
         const bool more = j + 1 < T;
         const int s2 = (j + 1) % C::kStages;
         if (more) {
@@ -277,9 +287,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           issue_s(0, s2);
           mma_commit(&ctl.s_full[0]);
         }
+        if (!(ok = mbar_wait(&ctl.p_half[1], j & 1, g))) break;
+        tc_fence_after();
+        issue_pv(1, s, j > 0, 0);
         if (!(ok = mbar_wait(&ctl.p_full[1], j & 1, g))) break;
         tc_fence_after();
-        issue_pv(1, s, j > 0);
+        issue_pv(1, s, j > 0, 1);
         mma_commit(&ctl.kv_empty[s]);
         if (more) {
           issue_s(1, s2);
@@ -345,6 +358,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
       const float2 c2 = make_float2(c, c), nmu2 = make_float2(-mu, -mu);
+      // The MMA warp starts P V on the first 64 keys as soon as their P is in
+      // TMEM (p_half), while this warpgroup computes the second half.
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         uint32_t pk[32];
@@ -353,21 +368,28 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         else
           exp_pack32<true, C::kEmuPairs>(&sr[64 * hf], c2, nmu2, acc, pk);
         tmem_st32(sreg + C::kPOff + 32 * hf, pk);
+        if (hf == 0) {
+          // The accumulator holds P V of earlier tiles (complete: the commit
+          // that signalled S_t came after them); rescale it where the
+          // reference moved, before any P V of this tile is issued.
+          if (__any_sync(0xffffffffu, grow && j > 0)) {
+#pragma unroll
+            for (int cc = 0; cc < D / 32; ++cc) {
+              uint32_t o[32];
+              tmem_ld32(oreg + cc * 32, o);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+              tmem_st32(oreg + cc * 32, o);
+            }
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.p_half[t]);
+        }
       }
       const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
       l += (a01.x + a01.y) + (a23.x + a23.y);
-      // The accumulator holds P V of earlier tiles (complete: the commit that
-      // signalled S_t came after them); rescale it where the reference moved.
-      if (__any_sync(0xffffffffu, grow && j > 0)) {
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(oreg + cc * 32, o);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-          tmem_st32(oreg + cc * 32, o);
-        }
-      }
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
