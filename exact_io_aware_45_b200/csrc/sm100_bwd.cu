@@ -90,7 +90,7 @@ struct Cfg {
 struct alignas(16) Ctl {
   uint64_t kv_full;
   uint64_t qdo_full[3], qdo_empty[3];
-  uint64_t sp_full[2], p_ready, dq_full, dq_free, acc_done;
+  uint64_t sp_full[2], p_ready[2], dq_full, dq_free, acc_done;
   uint32_t tmem_base;
   int abort;
   int nq;                      // visible query tiles per query head
@@ -152,7 +152,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
     }
     mbar_init(&ctl.sp_full[0], 1);
     mbar_init(&ctl.sp_full[1], 1);
-    mbar_init(&ctl.p_ready, C::kSoftWarps);
+    mbar_init(&ctl.p_ready[0], C::kSoftWarps);
+    mbar_init(&ctl.p_ready[1], C::kSoftWarps);
     mbar_init(&ctl.dq_full, 1);
     mbar_init(&ctl.dq_free, 4);
     mbar_init(&ctl.acc_done, 1);
@@ -184,6 +185,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   const int nq = ctl.nq;
   const int n_items = nq * grp;
   const Guard g{&ctl.abort, p.err};
+  constexpr int kChunks = MQ / 32 / (C::kSoftWarps / 4);   // 32-column chunks per softmax warp
+  static_assert(kChunks == 2, "the MMA warp waits on two chunk steps per item");
   // item i -> (query head, first query row)
   auto item_bh = [&](int i) { return b * p.Hq + hk * grp + i / nq; };
   auto item_q0 = [&](int i) { return static_cast<int>(ctl.qtiles[i % nq]) * MQ; };
@@ -255,20 +258,31 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
                  sdesc_sw128(ds_ + (kk >> 2) * C::kQBlock + (kk & 3) * 32, 16, 1024), idSP,
                  kk > 0);
       };
-      auto issue_dv = [&](int i) {  // dV += P^T dO_i (P^T bf16 in the S columns)
+      // dV += P^T dO_i and dK += dS^T Q_i over the query columns the softmax
+      // warps finished in chunk step `st` (32-column chunk cc = h * kChunks + st
+      // of each column half h; 16-query k-steps 2cc and 2cc + 1).
+      auto issue_dv = [&](int i, int st) {  // P^T bf16 in the S columns
         const uint32_t dos = dostage(i);
 #pragma unroll
-        for (int kk = 0; kk < MQ / 16; ++kk)
-          mma_ts(tm + C::kDV, tm + s_col(i) + (kk >> 1) * 32 + (kk & 1) * 8,
-                 sdesc_sw128(dos + kk * 2048, C::kQBlock, 1024), idKV, (i > 0 || kk > 0));
+        for (int h = 0; h < C::kSoftWarps / 4; ++h)
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int kk = 2 * (h * kChunks + st) + k2;
+            mma_ts(tm + C::kDV, tm + s_col(i) + (kk >> 1) * 32 + (kk & 1) * 8,
+                   sdesc_sw128(dos + kk * 2048, C::kQBlock, 1024), idKV, (i > 0 || kk > 0));
+          }
       };
-      auto issue_dk = [&](int i) {  // dK += dS^T Q_i
+      auto issue_dk = [&](int i, int st) {
         const uint32_t qs = qstage(i), dsb = dsbuf(i);
 #pragma unroll
-        for (int kk = 0; kk < MQ / 16; ++kk)
-          mma_ss(tm + C::kDK,
-                 sdesc_sw128(dsb + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(qs + kk * 2048, C::kQBlock, 1024), idKV, (i > 0 || kk > 0));
+        for (int h = 0; h < C::kSoftWarps / 4; ++h)
+#pragma unroll
+          for (int k2 = 0; k2 < 2; ++k2) {
+            const int kk = 2 * (h * kChunks + st) + k2;
+            mma_ss(tm + C::kDK,
+                   sdesc_sw128(dsb + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
+                   sdesc_sw128(qs + kk * 2048, C::kQBlock, 1024), idKV, (i > 0 || kk > 0));
+          }
       };
       auto issue_dq = [&](int i) {  // dQ_i^T = K^T dS_i^T (d = 128) or dQ_i = dS_i K (d = 64)
         const uint32_t dsb = dsbuf(i);
@@ -300,10 +314,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           mma_commit(&ctl.sp_full[1]);
         }
         for (int i = 0; ok && i < n_items; ++i) {
-          if (!(ok = mbar_wait(&ctl.p_ready, i & 1, g))) break;
+          // d = 128: one signal per item (per-chunk signals measured slower)
+          if (!(ok = mbar_wait(&ctl.p_ready[1], i & 1, g))) break;
           tc_fence_after();
-          issue_dv(i);
-          issue_dk(i);
+          issue_dv(i, 0);
+          issue_dv(i, 1);
+          issue_dk(i, 0);
+          issue_dk(i, 1);
           mma_commit(&ctl.qdo_empty[i % C::kStages]);
           issue_dq(i);
           mma_commit(&ctl.dq_full);
@@ -319,9 +336,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
         }
       } else {
         for (int i = 0; ok && i < n_items; ++i) {
-          if (!(ok = mbar_wait(&ctl.p_ready, i & 1, g))) break;
+          if (!(ok = mbar_wait(&ctl.p_ready[0], i & 1, g))) break;
           tc_fence_after();
-          issue_dv(i);
+          issue_dv(i, 0);
+          issue_dk(i, 0);
+          if (!(ok = mbar_wait(&ctl.p_ready[1], i & 1, g))) break;
+          tc_fence_after();
+          issue_dv(i, 1);
           if (i + 1 < n_items) {
             if (!(ok = wait_q(i + 1))) break;
             tc_fence_after();
@@ -329,7 +350,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
             issue_dp(i + 1);
             mma_commit(&ctl.sp_full[0]);
           }
-          issue_dk(i);
+          issue_dk(i, 1);
           mma_commit(&ctl.qdo_empty[i % C::kStages]);
           if (i > 0 && !(ok = mbar_wait(&ctl.dq_free, (i - 1) & 1, g))) break;
           tc_fence_after();
@@ -346,7 +367,6 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
     // query columns and warps 8-11 the second half; with 4, warps 4-7 take all.
     const int wq = warp & 3;
     const int half = (warp - 4) >> 2;
-    constexpr int kChunks = MQ / 32 / (C::kSoftWarps / 4);   // 32-column chunks per warp
     const int r = wq * 32 + lane;                 // key row inside the tile
     const int kv = n0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
@@ -399,12 +419,17 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           uint4 v = make_uint4(dk[k * 4 + 0], dk[k * 4 + 1], dk[k * 4 + 2], dk[k * 4 + 3]);
           *reinterpret_cast<uint4*>(dsrow + blk * (kBN * 128) + ((c16 ^ (r & 7)) << 4)) = v;
         }
+        // This chunk's P^T and dS^T are complete: for d = 64 the MMA warp
+        // may run the dV and dK steps over its query columns now; for d = 128
+        // it waits for the whole item (one signal after the last chunk).
+        if (C::kSoftWarps == 8 || ch == kChunks - 1) {
+          tmem_st_wait();
+          fence_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&ctl.p_ready[ch]);
+        }
       }
-      tmem_st_wait();
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.p_ready);
     }
     // ------------------------------------------------------------ dK, dV epilogue
     if (n_items > 0) {
