@@ -143,7 +143,7 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
                    const float* LSE, void* dQ, void* dK, void* dV, int B, int Hq, int Hkv,
                    int N, int d, float scale, int causal, const uint8_t* block_mask, int dtype,
                    int grad_dtype, void* workspace, size_t workspace_bytes, void* stream,
-                   int path, int stages) {
+                   int path, int stages, const int* cu = nullptr, int total = 0) {
   t_launches = 0;
   fa_status s = check_dims(B, Hq, Hkv, N, d, scale, causal, dtype);
   if (s != FA_OK) return s;
@@ -156,10 +156,14 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV, workspace};
   for (const void* q : ptrs)
     if (!aligned16(q)) return FA_ERR_INVALID_ARG;
-  if (workspace_bytes < fa_bwd_workspace_size(B, Hq, N, d)) return FA_ERR_INVALID_ARG;
+  const size_t need = cu ? fa_bwd_varlen_workspace_size(B, Hq, N, total, d)
+                        : fa_bwd_workspace_size(B, Hq, N, d);
+  if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
 
   Problem p;
   fill_common(p, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype, stream);
+  p.cu = cu;
+  p.total = total;
   p.Q = Q;
   p.K = K;
   p.V = V;
@@ -179,6 +183,8 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
 
   const bool tc_ok = sm100_bwd_supported(p);
   if (path == FA_PATH_TC && !tc_ok) return FA_ERR_UNSUPPORTED;
+  // variable-length batches run on the tensor-core kernels only
+  if (cu && (!tc_ok || path == FA_PATH_SIMT)) return FA_ERR_UNSUPPORTED;
   const bool use_tc = (path == FA_PATH_TC) || (path == FA_PATH_AUTO && tc_ok);
   // The tensor-core path accumulates dQ in fp32: straight into dQ for fp32
   // gradients, into the workspace accumulator (converted by the finalize
@@ -237,6 +243,83 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
 FA_STAGE_ENTRY(fa_bwd_preprocess, kPre)
 FA_STAGE_ENTRY(fa_bwd_main, kMain)
 FA_STAGE_ENTRY(fa_bwd_finalize, kFinal)
+
+size_t fa_bwd_varlen_workspace_size(int B, int Hq, int max_seqlen, int total, int d) {
+  if (B < 0 || Hq < 0 || max_seqlen < 0 || total < 0 || d < 0) return 0;
+  const size_t npad = (size_t)((max_seqlen + 127) / 128) * 128;
+  const size_t vec = align256(sizeof(float) * (size_t)B * Hq * npad);
+  const size_t acc = align256(sizeof(float) * (size_t)total * Hq * d);
+  return kErrBlock + 2 * vec + acc;
+}
+
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+// Checks shared by the variable-length entry points (they run on the
+// tensor-core kernels only: bf16, d in {64, 128}).
+fa_status check_varlen(const int* cu, int B, int max_seqlen, int total, int Hq, int Hkv, int d,
+                       float scale, int causal, int dtype) {
+  if (B < 0 || max_seqlen < 0 || total < 0 || Hq <= 0 || Hkv <= 0 || d <= 0)
+    return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0 || (causal != 0 && causal != 1)) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_F32 && dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (B > 0 && (!cu || (reinterpret_cast<uintptr_t>(cu) & 3u))) return FA_ERR_INVALID_ARG;
+  if (total > 0 && max_seqlen == 0) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_BF16 || (d != 64 && d != 128) || !(scale > 0.f)) return FA_ERR_UNSUPPORTED;
+  if ((long long)total * Hq >= (1ll << 31) || (long long)total * Hkv >= (1ll << 31) ||
+      (long long)B * Hq * (((long long)max_seqlen + 127) / 128 * 128) >= (1ll << 31))
+    return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                        const int* cu_seqlens, int B, int max_seqlen, int total, int Hq, int Hkv,
+                        int d, float scale, int causal, int dtype, void* workspace,
+                        void* stream) {
+  t_launches = 0;
+  fa_status s = check_varlen(cu_seqlens, B, max_seqlen, total, Hq, Hkv, d, scale, causal, dtype);
+  if (s != FA_OK) return s;
+  if (B == 0 || total == 0) return FA_OK;
+  if (!Q || !K || !V || !O || !LSE || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O) || !aligned16(LSE) ||
+      !aligned16(workspace))
+    return FA_ERR_INVALID_ARG;
+  Problem p;
+  fill_common(p, B, Hq, Hkv, max_seqlen, d, scale, causal, nullptr, dtype, stream);
+  p.cu = cu_seqlens;
+  p.total = total;
+  p.Q = Q;
+  p.K = K;
+  p.V = V;
+  p.Oout = O;
+  p.LSEout = LSE;
+  p.err = static_cast<unsigned*>(workspace);
+  if (!sm100_fwd_supported(p)) return FA_ERR_UNSUPPORTED;
+  return from_cuda(sm100_fwd(p));
+}
+
+fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O,
+                        const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                        const int* cu_seqlens, int B, int max_seqlen, int total, int Hq, int Hkv,
+                        int d, float scale, int causal, int dtype, int grad_dtype,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  t_launches = 0;
+  fa_status s = check_varlen(cu_seqlens, B, max_seqlen, total, Hq, Hkv, d, scale, causal, dtype);
+  if (s != FA_OK) return s;
+  if (grad_dtype != FA_F32 && grad_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
+  if (B == 0 || total == 0) return FA_OK;
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, Hq, Hkv, max_seqlen, d, scale, causal,
+                  nullptr, dtype, grad_dtype, workspace, workspace_bytes, stream, FA_PATH_TC,
+                  kAll, cu_seqlens, total);
+}
 
 fa_status fa_get_device_error(void* workspace, void* stream) {
   if (!workspace) return FA_ERR_INVALID_ARG;

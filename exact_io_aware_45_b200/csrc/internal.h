@@ -35,6 +35,10 @@ struct Problem {
   float* LSE2ws = nullptr;        // [B*Hq][Npad]  LSE * log2(e), +inf where empty
   float* dQacc = nullptr;         // [B*Hq][N][d]
   int Npad = 0;
+  // variable-length batch: sequence b is rows cu[b] .. cu[b+1]-1 of packed
+  // [total][H][d] tensors (LSE [Hq][total]); N is then the longest length
+  const int* cu = nullptr;
+  int total = 0;
   cudaStream_t stream = nullptr;
 };
 

@@ -138,6 +138,9 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(Problem p) {
 // P is 0), optionally zeroing the row of the fp32 dQ accumulator. TPR
 // threads share a row, each reading 16 bytes of O and of dO (VEC elements),
 // and the partial dots are summed with shuffles inside the TPR-lane group.
+// Variable-length batches (p.cu set): row r of (b, h) is token cu[b] + r of
+// the packed [total][Hq][d] tensors and LSE [Hq][total]; the vectors keep the
+// padded [B*Hq][Npad] layout (Npad from the longest sequence).
 template <typename T, int TPR>
 __global__ void __launch_bounds__(256) preprocess_kernel(Problem p, int zero_acc) {
   constexpr int VEC = 16 / sizeof(T);
@@ -150,8 +153,18 @@ __global__ void __launch_bounds__(256) preprocess_kernel(Problem p, int zero_acc
   const int row = live ? (int)(rowid % p.Npad) : p.N;
   const int d = p.d;
   float acc = 0.f;
-  if (live && row < p.N) {
-    const size_t off = ((size_t)bh * p.N + row) * d + (size_t)part * VEC;
+  int n_rows = p.N;
+  size_t row_off = (size_t)bh * p.N + row, lse_off = row_off;   // in units of d / of 1
+  if (p.cu && live) {
+    const int b = bh / p.Hq, h = bh % p.Hq;
+    const int s0 = min(max(p.cu[b], 0), p.total);
+    const int s1 = min(max(p.cu[b + 1], s0), p.total);
+    n_rows = min(s1 - s0, p.N);
+    row_off = (size_t)(s0 + row) * p.Hq + h;
+    lse_off = (size_t)h * p.total + s0 + row;
+  }
+  if (live && row < n_rows) {
+    const size_t off = row_off * d + (size_t)part * VEC;
     const uint4 ov = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.O) + off);
     const uint4 gv = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.dO) + off);
     const T* o = reinterpret_cast<const T*>(&ov);
@@ -168,8 +181,8 @@ __global__ void __launch_bounds__(256) preprocess_kernel(Problem p, int zero_acc
   for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
   if (live && part == 0) {
     float lse2 = INFINITY;
-    if (row < p.N) {
-      const float L = p.LSE[(size_t)bh * p.N + row];
+    if (row < n_rows) {
+      const float L = p.LSE[lse_off];
       if (L != -INFINITY) lse2 = L * kLog2e;
     }
     p.Dws[(size_t)bh * p.Npad + row] = acc;
@@ -410,8 +423,10 @@ cudaError_t simt_bwd_main(const Problem& p) {
 }
 
 cudaError_t dq_convert(const Problem& p) {
-  const size_t n = (size_t)p.B * p.Hq * p.N * p.d;  // d is a multiple of 16
+  const size_t rows = p.cu ? (size_t)p.total : (size_t)p.B * p.N;
+  const size_t n = rows * p.Hq * p.d;  // d is a multiple of 16
   const size_t n4 = n / 4;
+  if (n4 == 0) return cudaSuccess;
   const int blocks = (int)std::min<size_t>((n4 + 255) / 256, 148 * 16);
   if (p.grad_dtype == 0)
     dq_convert_kernel<float><<<blocks, 256, 0, p.stream>>>(p.dQacc, static_cast<float*>(p.dQ), n4);

@@ -110,6 +110,8 @@ struct BwdParams {
   int N, Npad, Hq, Hkv, nb, causal, grad_bf16, BHk;
   float c;                     // scale * log2(e)
   float scale;
+  const int* cu;               // variable-length batch: sequence offsets [B+1], or null
+  int total;                   // packed rows (variable-length batch)
 };
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -119,7 +121,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int D>
+template <int D, bool kVarlen>
 __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
   using C = Cfg<D>;
   constexpr int MQ = C::MQ;
@@ -142,7 +144,18 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   const int n0 = kb * kBN;
   const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
   const int grp = p.Hq / p.Hkv;
-  const int N = p.N;
+  // Dense: rows 0..N-1 of plane (b, head). Variable-length batch: sequence b
+  // is rows cu[b] .. cu[b+1]-1 of the packed tensors (planes are heads); key
+  // tiles past its end have nothing to do. Offsets are clamped to [0, total].
+  int N = p.N, row0 = 0;
+  if constexpr (kVarlen) {
+    const int s0 = min(max(p.cu[b], 0), p.total);
+    const int s1 = min(max(p.cu[b + 1], s0), p.total);
+    N = min(s1 - s0, p.N);
+    if (n0 >= N) return;
+    row0 = s0;
+  }
+  const int kplane = kVarlen ? hk : bhk;
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl.kv_full, 1);
@@ -189,6 +202,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   static_assert(kChunks == 2, "the MMA warp waits on two chunk steps per item");
   // item i -> (query head, first query row)
   auto item_bh = [&](int i) { return b * p.Hq + hk * grp + i / nq; };
+  // TMA plane of item i's Q / dO / dQ rows
+  auto item_plane = [&](int i) { return kVarlen ? hk * grp + i / nq : item_bh(i); };
   auto item_q0 = [&](int i) { return static_cast<int>(ctl.qtiles[i % nq]) * MQ; };
   // TMEM columns of item i
   auto s_col = [&](int i) { return (i & 1) ? C::kS1 : C::kS0; };
@@ -204,20 +219,22 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       prefetch_tmap(&p.tv);
       mbar_expect_tx(&ctl.kv_full, 2 * C::kKVBytes);
       for (int cb = 0; cb < D / 64; ++cb) {
-        tma_load_3d(base + C::kOffK + cb * kBN * 128, &p.tk, &ctl.kv_full, cb * 64, n0, bhk);
-        tma_load_3d(base + C::kOffV + cb * kBN * 128, &p.tv, &ctl.kv_full, cb * 64, n0, bhk);
+        tma_load_3d(base + C::kOffK + cb * kBN * 128, &p.tk, &ctl.kv_full, cb * 64, row0 + n0,
+                    kplane);
+        tma_load_3d(base + C::kOffV + cb * kBN * 128, &p.tv, &ctl.kv_full, cb * 64, row0 + n0,
+                    kplane);
       }
       int issued = 0;
       for (int i = 0; i < n_items; ++i) {
         const int s = i % C::kStages;
         if (i >= C::kStages && !mbar_wait(&ctl.qdo_empty[s], ((i / C::kStages) - 1) & 1, g)) break;
-        const int bh = item_bh(i), q0 = item_q0(i);
+        const int bh = item_bh(i), q0 = item_q0(i), pl = item_plane(i);
         mbar_expect_tx(&ctl.qdo_full[s], 2 * C::kQBytes + 2 * MQ * 4);
         for (int cb = 0; cb < D / 64; ++cb) {
           tma_load_3d(base + C::kOffQ + s * C::kQBytes + cb * C::kQBlock, &p.tq,
-                      &ctl.qdo_full[s], cb * 64, q0, bh);
+                      &ctl.qdo_full[s], cb * 64, row0 + q0, pl);
           tma_load_3d(base + C::kOffDO + s * C::kQBytes + cb * C::kQBlock, &p.tdo,
-                      &ctl.qdo_full[s], cb * 64, q0, bh);
+                      &ctl.qdo_full[s], cb * 64, row0 + q0, pl);
         }
         const size_t vo = (size_t)bh * p.Npad + q0;
         bulk_load(vec + (s * 2 + 0) * MQ, p.lse2 + vo, MQ * 4, &ctl.qdo_full[s]);
@@ -437,7 +454,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       tc_fence_after();
     }
     const bool valid = kv < N;
-    const size_t orow = ((size_t)bhk * N + (valid ? kv : 0)) * D;
+    // dK, dV rows: [B][Hkv][N][d] (dense) or [total][Hkv][d] (variable-length)
+    const size_t orow = kVarlen ? ((size_t)(row0 + (valid ? kv : 0)) * p.Hkv + hk) * D
+                                : ((size_t)bhk * N + (valid ? kv : 0)) * D;
     // 8 softmax warps: warps 4-7 store dK, warps 8-11 dV; 4: warps 4-7 both.
 #pragma unroll 1
     for (int which = (C::kSoftWarps == 8) ? half : 0;
@@ -491,7 +510,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.dq_free);
-      const int bh = item_bh(i), q0 = item_q0(i);
+      const int pl = item_plane(i), q0 = row0 + item_q0(i);
       if constexpr (D == 128) {
         // lane = head-dim column d = 32*wq + lane; v[q] for q = 0..63. Two
         // 16 KB halves: warps 0-1 stage d 0..63, then warps 2-3 stage 64..127.
@@ -510,8 +529,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           }
           named_sync(1, 128);
           if (leader) {
-            tma_reduce_add_3d(&p.tdq, stg, (2 * hf) * 32, q0, bh);
-            tma_reduce_add_3d(&p.tdq, stg + C::kStgBox, (2 * hf + 1) * 32, q0, bh);
+            tma_reduce_add_3d(&p.tdq, stg, (2 * hf) * 32, q0, pl);
+            tma_reduce_add_3d(&p.tdq, stg + C::kStgBox, (2 * hf + 1) * 32, q0, pl);
             bulk_commit();
           }
         }
@@ -534,7 +553,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
         if (leader) {
 #pragma unroll
           for (int bx = 0; bx < D / 32; ++bx)
-            tma_reduce_add_3d(&p.tdq, stg + bx * C::kStgBox, bx * 32, q0, bh);
+            tma_reduce_add_3d(&p.tdq, stg + bx * C::kStgBox, bx * 32, q0, pl);
           bulk_commit();
         }
       }
@@ -558,12 +577,12 @@ cudaError_t launch(const Problem& pr) {
   const uint64_t BHq = (uint64_t)pr.B * pr.Hq, BHk = (uint64_t)pr.B * pr.Hkv;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_tmap_3d(&kp.tq, pr.Q, bf, 2, D, pr.N, BHq, 64, C::MQ, sw) ||
-      !make_tmap_3d(&kp.tdo, pr.dO, bf, 2, D, pr.N, BHq, 64, C::MQ, sw) ||
-      !make_tmap_3d(&kp.tk, pr.K, bf, 2, D, pr.N, BHk, 64, kBN, sw) ||
-      !make_tmap_3d(&kp.tv, pr.V, bf, 2, D, pr.N, BHk, 64, kBN, sw) ||
-      !make_tmap_3d(&kp.tdq, pr.dQacc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, D, pr.N, BHq, 32,
-                    C::MQ, sw))
+  if (!make_seq_tmap(&kp.tq, pr, pr.Q, bf, 2, pr.Hq, 64, C::MQ, sw) ||
+      !make_seq_tmap(&kp.tdo, pr, pr.dO, bf, 2, pr.Hq, 64, C::MQ, sw) ||
+      !make_seq_tmap(&kp.tk, pr, pr.K, bf, 2, pr.Hkv, 64, kBN, sw) ||
+      !make_seq_tmap(&kp.tv, pr, pr.V, bf, 2, pr.Hkv, 64, kBN, sw) ||
+      !make_seq_tmap(&kp.tdq, pr, pr.dQacc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, pr.Hq, 32, C::MQ,
+                     sw))
     return cudaErrorInvalidValue;
   kp.lse2 = pr.LSE2ws;
   kp.dvec = pr.Dws;
@@ -580,17 +599,25 @@ cudaError_t launch(const Problem& pr) {
   kp.grad_bf16 = pr.grad_dtype == 1;
   kp.c = pr.scale * kLog2e;
   kp.scale = pr.scale;
+  kp.cu = pr.cu;
+  kp.total = pr.total;
   const size_t smem = sizeof(Ctl) + 1024 + C::kOffEnd;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(bwd_kernel<D, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(bwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   kp.BHk = (int)BHk;
   dim3 grid((unsigned)(BHk * pr.nb));
-  bwd_kernel<D><<<grid, C::kThreads, smem, pr.stream>>>(kp);
+  if (pr.cu)
+    bwd_kernel<D, true><<<grid, C::kThreads, smem, pr.stream>>>(kp);
+  else
+    bwd_kernel<D, false><<<grid, C::kThreads, smem, pr.stream>>>(kp);
   count_launch();
   return cudaGetLastError();
 }

@@ -431,5 +431,24 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
                   uint64_t cols, uint64_t rows, uint64_t planes, uint32_t box_cols,
                   uint32_t box_rows, CUtensorMapSwizzle swz);
+// As make_tmap_3d with explicit row and plane strides (in elements), e.g. the
+// packed [total][H][d] layout of variable-length batches: rows = tokens
+// (stride H*d), planes = heads (stride d).
+bool make_tmap_3d_strided(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                          int elem_bytes, uint64_t cols, uint64_t rows, uint64_t planes,
+                          uint64_t row_stride, uint64_t plane_stride, uint32_t box_cols,
+                          uint32_t box_rows, CUtensorMapSwizzle swz);
+// The map of a [B][H][N][cols] tensor (dense) or of a packed [total][H][cols]
+// one (variable-length, p.cu set); rows of the box run over N or tokens.
+inline bool make_seq_tmap(CUtensorMap* m, const Problem& p, const void* base,
+                          CUtensorMapDataType dt, int elem_bytes, int H, uint32_t box_cols,
+                          uint32_t box_rows, CUtensorMapSwizzle swz) {
+  const uint64_t d = (uint64_t)p.d;
+  if (p.cu)
+    return make_tmap_3d_strided(m, base, dt, elem_bytes, d, (uint64_t)p.total, (uint64_t)H,
+                                (uint64_t)H * d, d, box_cols, box_rows, swz);
+  return make_tmap_3d(m, base, dt, elem_bytes, d, (uint64_t)p.N, (uint64_t)p.B * H, box_cols,
+                      box_rows, swz);
+}
 
 }  // namespace fa

@@ -94,6 +94,8 @@ struct FwdParams {
   unsigned* err;
   int N, Hq, Hkv, nb, nblk, causal, BH;
   float c;                   // scale * log2(e)
+  const int* cu;             // variable-length batch: sequence offsets [B+1], or null
+  int total;                 // packed rows (variable-length batch)
 };
 
 // 32 pairs of scores -> p = 2^(s*c - mu) packed to bf16 pairs, with the
@@ -124,7 +126,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int D>
+template <int D, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -146,7 +148,20 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   const int bhk = b * p.Hkv + h / (p.Hq / p.Hkv);
   const int q0 = blk * 2 * kBM;
   const int qb0 = 2 * blk, qb1 = 2 * blk + 1;   // 128-row mask blocks of the two tiles
-  const int N = p.N;
+  // Dense: rows 0..N-1 of plane (b, h). Variable-length batch: sequence b is
+  // rows cu[b] .. cu[b+1]-1 of the packed tensors (planes are heads); blocks
+  // past its end have nothing to do. Offsets are clamped to [0, total].
+  int N = p.N, nb = p.nb, row0 = 0, qplane = bh, kplane = bhk;
+  if constexpr (kVarlen) {
+    const int s0 = min(max(p.cu[b], 0), p.total);
+    const int s1 = min(max(p.cu[b + 1], s0), p.total);
+    N = min(s1 - s0, p.N);
+    if (q0 >= N) return;
+    nb = (N + kBN - 1) / kBN;
+    row0 = s0;
+    qplane = h;
+    kplane = h / (p.Hq / p.Hkv);
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl.q_full, 1);
@@ -170,14 +185,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   }
   if (warp == 3) {
     // Key tiles either query tile can see, in increasing order.
-    const int kb_end = p.causal ? min(p.nb, qb1 + 1) : p.nb;
+    const int kb_end = p.causal ? min(nb, qb1 + 1) : nb;
     int count = 0;
     for (int kb0 = 0; kb0 < kb_end; kb0 += 32) {
       const int kb = kb0 + lane;
       bool a0 = false, a1 = false;
       if (kb < kb_end) {
         a0 = (!p.mask || p.mask[(size_t)qb0 * p.nb + kb]) && (!p.causal || kb <= qb0);
-        a1 = qb1 < p.nb && (!p.mask || p.mask[(size_t)qb1 * p.nb + kb]) &&
+        a1 = qb1 < nb && (!p.mask || p.mask[(size_t)qb1 * p.nb + kb]) &&
              (!p.causal || kb <= qb1);
       }
       const bool act = a0 || a1;
@@ -208,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       for (int t = 0; t < 2; ++t)
         for (int cb = 0; cb < C::kColBlocks; ++cb)
           tma_load_3d(tiles_base + C::kOffQ + t * C::kQBytes + cb * C::kBlockBytes, &p.tq,
-                      &ctl.q_full, cb * 64, q0 + t * kBM, bh);
+                      &ctl.q_full, cb * 64, row0 + q0 + t * kBM, qplane);
       int issued = 0;
       for (int j = 0; j < T; ++j) {
         const int s = j % C::kStages;
@@ -218,11 +233,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         mbar_expect_tx(&ctl.k_full[s], C::kTileBytes);
         for (int cb = 0; cb < C::kColBlocks; ++cb)
           tma_load_3d(tiles_base + C::kOffK + s * C::kTileBytes + cb * C::kBlockBytes, &p.tk,
-                      &ctl.k_full[s], cb * 64, kb * kBN, bhk);
+                      &ctl.k_full[s], cb * 64, row0 + kb * kBN, kplane);
         mbar_expect_tx(&ctl.v_full[s], C::kTileBytes);
         for (int cb = 0; cb < C::kColBlocks; ++cb)
           tma_load_3d(tiles_base + C::kOffV + s * C::kTileBytes + cb * C::kBlockBytes, &p.tv,
-                      &ctl.v_full[s], cb * 64, kb * kBN, bhk);
+                      &ctl.v_full[s], cb * 64, row0 + kb * kBN, kplane);
         issued = j + 1;
       }
       // Every issued copy has landed before the CTA may exit.
@@ -402,7 +417,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     }
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
     const bool valid = row < N;
-    __nv_bfloat16* out = p.O + ((size_t)bh * N + (valid ? row : 0)) * D;
+    // O rows: [B][H][N][d] (dense) or [total][H][d] (variable-length)
+    const size_t o_base = kVarlen ? ((size_t)row0 * p.Hq + h) * D : (size_t)bh * p.N * D;
+    const size_t o_rs = kVarlen ? (size_t)p.Hq * D : (size_t)D;
+    const size_t lse_base = kVarlen ? (size_t)h * p.total + row0 : (size_t)bh * p.N;
+    __nv_bfloat16* out = p.O + o_base + (size_t)(valid ? row : 0) * o_rs;
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t o[32];
@@ -423,7 +442,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         for (int i = 0; i < 4; ++i) dst[i] = v[i];
       }
     }
-    if (valid) p.LSE[(size_t)bh * N + row] = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+    if (valid) p.LSE[lse_base + row] = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
   }
 
   tc_fence_before();
@@ -439,12 +458,12 @@ cudaError_t launch(const Problem& pr) {
   using C = Cfg<D>;
   FwdParams kp;
   memset(&kp, 0, sizeof(kp));
-  const uint64_t BHq = (uint64_t)pr.B * pr.Hq, BHk = (uint64_t)pr.B * pr.Hkv;
+  const uint64_t BHq = (uint64_t)pr.B * pr.Hq;
   const auto bf = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
-  if (!make_tmap_3d(&kp.tq, pr.Q, bf, 2, D, pr.N, BHq, 64, kBM, sw) ||
-      !make_tmap_3d(&kp.tk, pr.K, bf, 2, D, pr.N, BHk, 64, kBN, sw) ||
-      !make_tmap_3d(&kp.tv, pr.V, bf, 2, D, pr.N, BHk, 64, kBN, sw))
+  if (!make_seq_tmap(&kp.tq, pr, pr.Q, bf, 2, pr.Hq, 64, kBM, sw) ||
+      !make_seq_tmap(&kp.tk, pr, pr.K, bf, 2, pr.Hkv, 64, kBN, sw) ||
+      !make_seq_tmap(&kp.tv, pr, pr.V, bf, 2, pr.Hkv, 64, kBN, sw))
     return cudaErrorInvalidValue;
   kp.O = static_cast<__nv_bfloat16*>(pr.Oout);
   kp.LSE = pr.LSEout;
@@ -457,17 +476,25 @@ cudaError_t launch(const Problem& pr) {
   kp.nblk = (pr.N + 2 * kBM - 1) / (2 * kBM);
   kp.causal = pr.causal;
   kp.c = pr.scale * kLog2e;
+  kp.cu = pr.cu;
+  kp.total = pr.total;
   const size_t smem = sizeof(Ctl) + 1024 + C::kOffEnd;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D>,
+    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, false>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   kp.BH = (int)BHq;
   dim3 grid((unsigned)(BHq * kp.nblk));
-  fwd_kernel<D><<<grid, kThreads, smem, pr.stream>>>(kp);
+  if (pr.cu)
+    fwd_kernel<D, true><<<grid, kThreads, smem, pr.stream>>>(kp);
+  else
+    fwd_kernel<D, false><<<grid, kThreads, smem, pr.stream>>>(kp);
   count_launch();
   return cudaGetLastError();
 }

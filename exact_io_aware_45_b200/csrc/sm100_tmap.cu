@@ -31,6 +31,22 @@ EncodeTiled encode_fn() {
 
 }  // namespace
 
+bool make_tmap_3d_strided(CUtensorMap* m, const void* base, CUtensorMapDataType dt,
+                          int elem_bytes, uint64_t cols, uint64_t rows, uint64_t planes,
+                          uint64_t row_stride, uint64_t plane_stride, uint32_t box_cols,
+                          uint32_t box_rows, CUtensorMapSwizzle swz) {
+  EncodeTiled fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {cols, rows, planes};
+  cuuint64_t strides[2] = {row_stride * (uint64_t)elem_bytes, plane_stride * (uint64_t)elem_bytes};
+  cuuint32_t box[3] = {box_cols, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes,
                   uint64_t cols, uint64_t rows, uint64_t planes, uint32_t box_cols,
                   uint32_t box_rows, CUtensorMapSwizzle swz) {

@@ -26,7 +26,8 @@ PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
 # every symbol include/fa.h declares
 EXPORTS = ("fa_status_string", "fa_version", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
            "fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_preprocess", "fa_bwd_main",
-           "fa_bwd_finalize", "fa_last_launch_count", "fa_get_device_error", "fa_exp2_fma")
+           "fa_bwd_finalize", "fa_last_launch_count", "fa_get_device_error", "fa_exp2_fma",
+           "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_size")
 
 _lib = None
 
@@ -71,6 +72,14 @@ def lib() -> ctypes.CDLL:
         L.fa_get_device_error.argtypes = [_P, _P]
         L.fa_exp2_fma.argtypes = [_P, _P, ctypes.c_longlong, _P]
         L.fa_exp2_fma.restype = _I
+        L.fa_fwd_varlen.argtypes = [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I, _I,
+                                    _P, _P]
+        L.fa_fwd_varlen.restype = _I
+        L.fa_bwd_varlen.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
+                                    _I, _F, _I, _I, _I, _P, _S, _P]
+        L.fa_bwd_varlen.restype = _I
+        L.fa_bwd_varlen_workspace_size.argtypes = [_I, _I, _I, _I, _I]
+        L.fa_bwd_varlen_workspace_size.restype = _S
         _lib = L
     return _lib
 
@@ -131,6 +140,18 @@ def fa_get_device_error(workspace_ptr: int, stream_ptr: int) -> int:
 
 def fa_exp2_fma(x_ptr: int, y_ptr: int, n: int, stream_ptr: int) -> int:
     return lib().fa_exp2_fma(x_ptr, y_ptr, n, stream_ptr)
+
+
+def fa_fwd_varlen(*args) -> int:
+    return lib().fa_fwd_varlen(*args)
+
+
+def fa_bwd_varlen(*args) -> int:
+    return lib().fa_bwd_varlen(*args)
+
+
+def fa_bwd_varlen_workspace_size(B, Hq, max_seqlen, total, d) -> int:
+    return lib().fa_bwd_varlen_workspace_size(B, Hq, max_seqlen, total, d)
 
 
 # ------------------------------------------------------------------ torch helpers
@@ -210,6 +231,51 @@ def backward(q, k, v, o, do, lse, scale: Optional[float] = None, causal: bool = 
                   _dtype_code(q.dtype), _dtype_code(gdt), _ptr(ws), ws.numel(), _stream(),
                   int(path))
     _check(s, "fa_bwd")
+    return dq, dk, dv
+
+
+def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, scale: Optional[float] = None,
+                   causal: bool = False, out=None, lse=None, workspace=None):
+    """Variable-length batch: q [total, Hq, d], k/v [total, Hkv, d] (bf16,
+    sequences packed back to back), cu_seqlens int32 CUDA tensor [B + 1].
+    Returns O [total, Hq, d] and LSE [Hq, total]."""
+    import torch
+    total, Hq, d = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((Hq, total), dtype=torch.float32, device=q.device) if lse is None else lse
+    ws = new_workspace(fa_fwd_workspace_size(), q.device) if workspace is None else workspace
+    s = fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), _ptr(cu_seqlens), B,
+                      int(max_seqlen), total, Hq, Hkv, d, float(scale), int(bool(causal)),
+                      _dtype_code(q.dtype), _ptr(ws), _stream())
+    _check(s, "fa_fwd_varlen")
+    return o, l
+
+
+def backward_varlen(q, k, v, o, do, lse, cu_seqlens, max_seqlen: int,
+                    scale: Optional[float] = None, causal: bool = False, grad_dtype=None,
+                    workspace=None):
+    """dQ, dK, dV of a variable-length batch (layouts as forward_varlen)."""
+    import torch
+    total, Hq, d = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    gdt = torch.float32 if grad_dtype is None else grad_dtype
+    dq = torch.empty(q.shape, dtype=gdt, device=q.device)
+    dk = torch.empty(k.shape, dtype=gdt, device=q.device)
+    dv = torch.empty(v.shape, dtype=gdt, device=q.device)
+    nbytes = fa_bwd_varlen_workspace_size(B, Hq, int(max_seqlen), total, d)
+    ws = new_workspace(nbytes, q.device) if workspace is None else workspace
+    s = fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                      _ptr(dk), _ptr(dv), _ptr(cu_seqlens), B, int(max_seqlen), total, Hq, Hkv,
+                      d, float(scale), int(bool(causal)), _dtype_code(q.dtype), _dtype_code(gdt),
+                      _ptr(ws), ws.numel(), _stream())
+    _check(s, "fa_bwd_varlen")
     return dq, dk, dv
 
 

@@ -182,3 +182,39 @@ def flops(w_or_dims, N=None, causal=None, mask=None, backward=False) -> float:
         B, Hq, d = w_or_dims
     per = 10 * d if backward else 4 * d
     return float(per) * allowed_count(N, causal, mask) * B * Hq
+
+
+def varlen_case(lengths, Hq: int, Hkv: int, d: int, seed: int = 0):
+    """A variable-length batch: sequences of the given lengths packed back to
+    back. ``default_rng(seed)`` draws Q, K, V, dO in that order as float32
+    standard normals of shape [total, H, d] (K and V with Hkv heads), each
+    rounded to bfloat16. Returns the arrays, the int32 offsets cu [B + 1]
+    and max(lengths)."""
+    lengths = [int(n) for n in lengths]
+    cu = np.zeros(len(lengths) + 1, dtype=np.int32)
+    cu[1:] = np.cumsum(lengths)
+    total = int(cu[-1])
+    rng = np.random.default_rng(seed)
+    out = {}
+    for name, h in (("q", Hq), ("k", Hkv), ("v", Hkv), ("do", Hq)):
+        out[name] = bf16_round(rng.standard_normal((total, h, d), dtype=np.float32))
+    out["cu"] = cu
+    out["max_seqlen"] = max(lengths) if lengths else 0
+    return out
+
+
+def varlen_lengths(total_target: int, lo: int, hi: int, seed: int = 0):
+    """Seeded sequence lengths drawn uniformly from [lo, hi] until their sum
+    reaches total_target (the last one is cut so the sum is exact)."""
+    rng = np.random.default_rng(seed)
+    lengths, s = [], 0
+    while s < total_target:
+        n = int(min(rng.integers(lo, hi + 1), total_target - s))
+        lengths.append(n)
+        s += n
+    return lengths
+
+
+def varlen_allowed_count(lengths, causal: bool) -> int:
+    """Score elements a variable-length batch computes (per head)."""
+    return sum(allowed_count(n, causal, None) for n in lengths)

@@ -157,6 +157,39 @@ fa_status fa_bwd_finalize(const void* Q, const void* K, const void* V, const voi
                           void* workspace, size_t workspace_bytes, void* stream, int path);
 
 /*
+ * Variable-length (padding-free) batches. The glossary page ("Sequence Length
+ * Flexibility") names arbitrary sequence lengths without padding; these entry
+ * points take B sequences packed back to back:
+ *   Q, O, dO, dQ: [total][Hq][d]; K, V, dK, dV: [total][Hkv][d];
+ *   LSE: float [Hq][total];
+ *   cu_seqlens: device int32 [B + 1], cu_seqlens[0] = 0, non-decreasing,
+ *   cu_seqlens[B] = total; sequence b is rows cu_seqlens[b] .. cu_seqlens[b+1]-1
+ *   and attends only to itself (the causal flag is applied per sequence);
+ *   max_seqlen >= every length (it sizes the grid).
+ * Offsets are clamped to [0, total] on the device and a sequence longer than
+ * max_seqlen is cut to it, so inconsistent offsets give wrong results but no
+ * access outside the tensors. Tensor-core kernels only: dtype bf16, d in
+ * {64, 128}, scale > 0 (FA_ERR_UNSUPPORTED otherwise); no block mask. The
+ * workspace rules are those of fa_fwd / fa_bwd, with
+ * fa_bwd_varlen_workspace_size for the backward.
+ */
+fa_status fa_fwd_varlen(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                        const int* cu_seqlens, int B, int max_seqlen, int total, int Hq, int Hkv,
+                        int d, float scale, int causal, int dtype, void* workspace,
+                        void* stream);
+
+fa_status fa_bwd_varlen(const void* Q, const void* K, const void* V, const void* O,
+                        const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                        const int* cu_seqlens, int B, int max_seqlen, int total, int Hq, int Hkv,
+                        int d, float scale, int causal, int dtype, int grad_dtype,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace fa_bwd_varlen needs: the error-word block, D and the
+ * log2-scaled LSE (float [B*Hq][ceil(max_seqlen/128)*128] each) and the fp32
+ * dQ accumulator (float [total][Hq][d]). Returns 0 for negative sizes. */
+size_t fa_bwd_varlen_workspace_size(int B, int Hq, int max_seqlen, int total, int d);
+
+/*
  * fa_bwd_noalloc -- the backward pass for callers that cannot allocate.
  *
  * No passage of the FlashAttention pages corresponds to this entry point; it

@@ -241,3 +241,45 @@ def naive_forward_f32(Q2, K2, V2, scale):
     S = S - S.max(axis=1, keepdims=True)
     P = np.exp(S)
     return (P / P.sum(axis=1, keepdims=True)) @ V2.astype(np.float32)
+
+
+# ---------------------------------------------------------------- variable-length batches
+#
+# A packed batch of B sequences (glossary page, "Sequence Length Flexibility"):
+# sequence b is rows cu[b] .. cu[b+1]-1 of Q, K, V [total, H, d] and attends
+# only to itself. By definition it is the per-sequence attention above, so
+# the oracle applies forward / backward to each slice (as a batch of one) and
+# writes the results back in the packed layout; LSE is [Hq, total].
+
+def _seq(x, s0, s1):
+    """[s1 - s0, H, d] slice -> [1, H, n, d]."""
+    return np.ascontiguousarray(np.transpose(x[s0:s1], (1, 0, 2))[None])
+
+
+def forward_varlen(Q, K, V, cu, scale, causal=False):
+    total, Hq, d = Q.shape
+    O = np.zeros((total, Hq, d))
+    L = np.full((Hq, total), -np.inf)
+    for b in range(len(cu) - 1):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        if s1 == s0:
+            continue
+        Ob, Lb = forward(_seq(Q, s0, s1), _seq(K, s0, s1), _seq(V, s0, s1), scale, causal)
+        O[s0:s1] = np.transpose(Ob[0], (1, 0, 2))
+        L[:, s0:s1] = Lb[0]
+    return O, L
+
+
+def backward_varlen(Q, K, V, dO, cu, scale, causal=False):
+    dQ = np.zeros(Q.shape)
+    dK = np.zeros(K.shape)
+    dV = np.zeros(V.shape)
+    for b in range(len(cu) - 1):
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        if s1 == s0:
+            continue
+        g = backward(_seq(Q, s0, s1), _seq(K, s0, s1), _seq(V, s0, s1), _seq(dO, s0, s1), scale,
+                     causal)
+        for dst, src in zip((dQ, dK, dV), g):
+            dst[s0:s1] = np.transpose(src[0], (1, 0, 2))
+    return dQ, dK, dV
