@@ -55,7 +55,8 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama7b_causal",
-                    choices=[k for k, w in inputs.WORKLOADS.items() if w.backward])
+                    choices=[k for k, w in inputs.WORKLOADS.items() if w.backward] +
+                    [VARLEN_NAME])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -417,10 +418,118 @@ def run_ours(args):
     return 0
 
 
+# ---------------------------------------------------------------- variable-length batch
+
+VARLEN_NAME = "varlen_mix"
+VARLEN = dict(total=32768, lo=256, hi=4096, Hq=32, Hkv=32, d=128, causal=True)
+
+
+def run_varlen(args):
+    """One step = fa_fwd_varlen + fa_bwd_varlen on a packed batch of seeded
+    lengths (uniform in [256, 4096], 32768 tokens, 32 heads, d = 128, causal):
+    a padding-free training batch. Not the headline workload; its own line."""
+    import torch
+    from exact_io_aware_45_b200 import fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.lib()
+    c = VARLEN
+    lengths = inputs.varlen_lengths(c["total"], c["lo"], c["hi"], seed=0)
+    x = inputs.varlen_case(lengths, c["Hq"], c["Hkv"], c["d"], seed=rank)
+    bf = torch.bfloat16
+    q, k, v, do = (torch.from_numpy(x[n]).to(dev, bf).contiguous() for n in ("q", "k", "v", "do"))
+    cu = torch.from_numpy(x["cu"]).to(dev)
+    total, Hq, Hkv, d, B = c["total"], c["Hq"], c["Hkv"], c["d"], len(lengths)
+    maxlen = x["max_seqlen"]
+    scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    lse = torch.empty((Hq, total), dtype=torch.float32, device=dev)
+    dq, dk, dv = (torch.empty(t.shape, dtype=torch.float32, device=dev) for t in (q, k, v))
+    wsb = fa.fa_bwd_varlen_workspace_size(B, Hq, maxlen, total, d)
+    ws = fa.new_workspace(wsb, dev)
+    sp = torch.cuda.current_stream(dev).cuda_stream
+    P = lambda t: t.data_ptr()  # noqa: E731
+    fargs = (P(q), P(k), P(v), P(o), P(lse), P(cu), B, maxlen, total, Hq, Hkv, d, scale,
+             int(c["causal"]), fa.FA_BF16, P(ws), sp)
+    bargs = (P(q), P(k), P(v), P(o), P(do), P(lse), P(dq), P(dk), P(dv), P(cu), B, maxlen, total,
+             Hq, Hkv, d, scale, int(c["causal"]), fa.FA_BF16, fa.FA_F32, P(ws), wsb, sp)
+    stages = [("fwd", lambda: fa.fa_fwd_varlen(*fargs)), ("bwd", lambda: fa.fa_bwd_varlen(*bargs))]
+    allowed = inputs.varlen_allowed_count(lengths, c["causal"]) * Hq
+    fl = {"fwd": 4.0 * d * allowed, "bwd": 10.0 * d * allowed}
+    launches = 0
+
+    def step(evs=None):
+        n = 0
+        if evs is not None:
+            evs[0].record()
+        for i, (name, fn) in enumerate(stages):
+            st = fn()
+            if st != fa.FA_OK:
+                raise RuntimeError(f"{name}: {fa.status_string(st)}")
+            n += fa.fa_last_launch_count()
+            if evs is not None:
+                evs[i + 1].record()
+        return n
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    sampler.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(args.steps):
+        launches += step(evs[i])
+    t1.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    if fa.device_error(ws) != fa.FA_OK:
+        raise RuntimeError("device error word set")
+    ms = t0.elapsed_time(t1)
+    per = {name: statistics.mean(e[j].elapsed_time(e[j + 1]) for e in evs)
+           for j, (name, _) in enumerate(stages)}
+    value = (fl["fwd"] + fl["bwd"]) * args.steps * world / (ms / 1e3) / 1e12
+    peaks, kind = measured_peaks()
+    peak = (peaks or {}).get("bf16_tflops", FALLBACK_PEAK_TFLOPS)
+    dom = max(per, key=per.get)
+    ach = fl[dom] / (per[dom] / 1e3) / 1e12
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1) rounded to bf16; seeded lengths)",
+            "config": {"workload": f"{VARLEN_NAME}: {B} sequences, lengths uniform in "
+                                   f"[{c['lo']}, {c['hi']}], {total} tokens, Hq={Hq} Hkv={Hkv} "
+                                   f"d={d} causal bf16 fwd+bwd (padding-free)",
+                       "B": B, "total": total, "max_seqlen": maxlen, "Hq": Hq, "Hkv": Hkv,
+                       "d": d, "causal": c["causal"], "grad_dtype": "f32",
+                       "parallelism": f"replicas x{world} (independent batches)"},
+            "stages_ms": per,
+            "per_direction": {"fwd_tflops": fl["fwd"] / (per["fwd"] / 1e3) / 1e12,
+                              "bwd_tflops": fl["bwd"] / (per["bwd"] / 1e3) / 1e12},
+            "roofline": {"bound": "tensor", "kernel": dom, "achieved": ach, "peak": peak,
+                         "unit": "TFLOP/s", "frac": ach / peak,
+                         "peak_kind": f"{kind} burst bf16", "traffic": None},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": launches, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
+        if args.workload == VARLEN_NAME:
+            print(json.dumps({"impl": "reference", "unavailable": "the reference arm times the "
+                              "oracle on the headline workloads only"}))
+            return 0
         return run_reference(args)
+    if args.workload == VARLEN_NAME:
+        return run_varlen(args)
     return run_ours(args)
 
 
