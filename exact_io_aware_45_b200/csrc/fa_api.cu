@@ -143,7 +143,8 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
                    const float* LSE, void* dQ, void* dK, void* dV, int B, int Hq, int Hkv,
                    int N, int d, float scale, int causal, const uint8_t* block_mask, int dtype,
                    int grad_dtype, void* workspace, size_t workspace_bytes, void* stream,
-                   int path, int stages, const int* cu = nullptr, int total = 0) {
+                   int path, int stages, const int* cu = nullptr, int total = 0,
+                   int deterministic = 0) {
   t_launches = 0;
   fa_status s = check_dims(B, Hq, Hkv, N, d, scale, causal, dtype);
   if (s != FA_OK) return s;
@@ -185,20 +186,30 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   if (path == FA_PATH_TC && !tc_ok) return FA_ERR_UNSUPPORTED;
   // variable-length batches run on the tensor-core kernels only
   if (cu && (!tc_ok || path == FA_PATH_SIMT)) return FA_ERR_UNSUPPORTED;
+  // Deterministic gradients: the CUDA-core kernels use no atomics already; on
+  // the tensor-core path the main kernel skips dQ and the dQ kernel computes
+  // it per query tile.
+  const bool det_tc = deterministic && ((path == FA_PATH_TC) || (path == FA_PATH_AUTO && tc_ok));
+  if (det_tc && !sm100_dq_supported(p)) return FA_ERR_UNSUPPORTED;
+  p.no_dq = det_tc ? 1 : 0;
   const bool use_tc = (path == FA_PATH_TC) || (path == FA_PATH_AUTO && tc_ok);
   // The tensor-core path accumulates dQ in fp32: straight into dQ for fp32
   // gradients, into the workspace accumulator (converted by the finalize
   // stage) for bf16 gradients. The preprocess zeroes whichever it is.
-  const bool use_acc = use_tc && sm100_bwd_uses_dq_accumulator(p);
+  const bool use_acc = use_tc && !det_tc && sm100_bwd_uses_dq_accumulator(p);
   if (use_tc && !use_acc) p.dQacc = static_cast<float*>(dQ);
   cudaError_t e = cudaSuccess;
   if (stages & kPre) {
-    e = bwd_preprocess(p, use_tc);
+    e = bwd_preprocess(p, use_tc && !det_tc);
     if (e != cudaSuccess) return FA_ERR_CUDA;
   }
   if (stages & kMain) {
     e = use_tc ? sm100_bwd_main(p) : simt_bwd_main(p);
     if (e != cudaSuccess) return FA_ERR_CUDA;
+    if (det_tc) {
+      e = sm100_dq(p);
+      if (e != cudaSuccess) return FA_ERR_CUDA;
+    }
   }
   if ((stages & kFinal) && use_acc) {
     e = dq_convert(p);
@@ -243,6 +254,16 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
 FA_STAGE_ENTRY(fa_bwd_preprocess, kPre)
 FA_STAGE_ENTRY(fa_bwd_main, kMain)
 FA_STAGE_ENTRY(fa_bwd_finalize, kFinal)
+
+fa_status fa_bwd_deterministic(const void* Q, const void* K, const void* V, const void* O,
+                               const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                               int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                               const uint8_t* block_mask, int dtype, int grad_dtype,
+                               void* workspace, size_t workspace_bytes, void* stream, int path) {
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, Hq, Hkv, N, d, scale, causal, block_mask,
+                  dtype, grad_dtype, workspace, workspace_bytes, stream, path, kAll, nullptr, 0,
+                  1);
+}
 
 size_t fa_bwd_varlen_workspace_size(int B, int Hq, int max_seqlen, int total, int d) {
   if (B < 0 || Hq < 0 || max_seqlen < 0 || total < 0 || d < 0) return 0;

@@ -39,6 +39,8 @@ struct Problem {
   // [total][H][d] tensors (LSE [Hq][total]); N is then the longest length
   const int* cu = nullptr;
   int total = 0;
+  // backward main kernel: skip dQ (computed by the deterministic dQ kernel)
+  int no_dq = 0;
   cudaStream_t stream = nullptr;
 };
 
@@ -62,5 +64,8 @@ cudaError_t exp2_fma_eval(const float* x, float* y, long long n, cudaStream_t st
 bool sm100_bwd_supported(const Problem& p);
 bool sm100_bwd_uses_dq_accumulator(const Problem& p);
 cudaError_t sm100_bwd_main(const Problem& p);
+// Deterministic dQ (no atomics): one CTA per query tile. sm100_dq.cu
+bool sm100_dq_supported(const Problem& p);
+cudaError_t sm100_dq(const Problem& p);
 
 }  // namespace fa

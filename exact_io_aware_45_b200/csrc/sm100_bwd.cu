@@ -112,6 +112,7 @@ struct BwdParams {
   float scale;
   const int* cu;               // variable-length batch: sequence offsets [B+1], or null
   int total;                   // packed rows (variable-length batch)
+  int no_dq;                   // skip dQ (the deterministic dQ kernel computes it)
 };
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -339,13 +340,15 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           issue_dk(i, 0);
           issue_dk(i, 1);
           mma_commit(&ctl.qdo_empty[i % C::kStages]);
-          issue_dq(i);
-          mma_commit(&ctl.dq_full);
+          if (!p.no_dq) {
+            issue_dq(i);
+            mma_commit(&ctl.dq_full);
+          }
           if (i + 2 < n_items) {
             if (!(ok = wait_q(i + 2))) break;
             tc_fence_after();
             issue_dp(i + 2);
-            if (!(ok = mbar_wait(&ctl.dq_free, i & 1, g))) break;   // dQ(i) drained
+            if (!p.no_dq && !(ok = mbar_wait(&ctl.dq_free, i & 1, g))) break;   // dQ(i) drained
             tc_fence_after();
             issue_s(i + 2);
             mma_commit(&ctl.sp_full[i & 1]);
@@ -369,10 +372,12 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           }
           issue_dk(i, 1);
           mma_commit(&ctl.qdo_empty[i % C::kStages]);
-          if (i > 0 && !(ok = mbar_wait(&ctl.dq_free, (i - 1) & 1, g))) break;
-          tc_fence_after();
-          issue_dq(i);
-          mma_commit(&ctl.dq_full);
+          if (!p.no_dq) {
+            if (i > 0 && !(ok = mbar_wait(&ctl.dq_free, (i - 1) & 1, g))) break;
+            tc_fence_after();
+            issue_dq(i);
+            mma_commit(&ctl.dq_full);
+          }
         }
       }
       mma_commit(&ctl.acc_done);
@@ -502,7 +507,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
     const float sc = p.scale;
     // Every drain thread runs all iterations (waits return at once after an
     // abort), so the named barriers below always see all 128 threads.
-    for (int i = 0; i < n_items; ++i) {
+    const int n_drain = p.no_dq ? 0 : n_items;
+    for (int i = 0; i < n_drain; ++i) {
       mbar_wait(&ctl.dq_full, i & 1, g);
       tc_fence_after();
       uint32_t v[64];
@@ -601,6 +607,7 @@ cudaError_t launch(const Problem& pr) {
   kp.scale = pr.scale;
   kp.cu = pr.cu;
   kp.total = pr.total;
+  kp.no_dq = pr.no_dq;
   const size_t smem = sizeof(Ctl) + 1024 + C::kOffEnd;
   static bool attr_set = false;
   if (!attr_set) {

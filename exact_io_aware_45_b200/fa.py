@@ -27,7 +27,8 @@ PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
 EXPORTS = ("fa_status_string", "fa_version", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
            "fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_preprocess", "fa_bwd_main",
            "fa_bwd_finalize", "fa_last_launch_count", "fa_get_device_error", "fa_exp2_fma",
-           "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_size")
+           "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_size",
+           "fa_bwd_deterministic")
 
 _lib = None
 
@@ -63,10 +64,11 @@ def lib() -> ctypes.CDLL:
         L.fa_fwd.argtypes = _FWD_ARGS
         L.fa_fwd_ex.argtypes = _FWD_ARGS + [_I]
         L.fa_bwd.argtypes = _BWD_ARGS
-        for n in ("fa_bwd_ex", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finalize"):
+        for n in ("fa_bwd_ex", "fa_bwd_preprocess", "fa_bwd_main", "fa_bwd_finalize",
+                  "fa_bwd_deterministic"):
             getattr(L, n).argtypes = _BWD_ARGS + [_I]
         for n in ("fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_preprocess",
-                  "fa_bwd_main", "fa_bwd_finalize", "fa_get_device_error"):
+                  "fa_bwd_main", "fa_bwd_finalize", "fa_get_device_error", "fa_bwd_deterministic"):
             getattr(L, n).restype = _I
         L.fa_last_launch_count.restype = _I
         L.fa_get_device_error.argtypes = [_P, _P]
@@ -142,6 +144,10 @@ def fa_exp2_fma(x_ptr: int, y_ptr: int, n: int, stream_ptr: int) -> int:
     return lib().fa_exp2_fma(x_ptr, y_ptr, n, stream_ptr)
 
 
+def fa_bwd_deterministic(*args) -> int:
+    return lib().fa_bwd_deterministic(*args)
+
+
 def fa_fwd_varlen(*args) -> int:
     return lib().fa_fwd_varlen(*args)
 
@@ -213,9 +219,11 @@ def forward(q, k, v, scale: Optional[float] = None, causal: bool = False, block_
 
 
 def backward(q, k, v, o, do, lse, scale: Optional[float] = None, causal: bool = False,
-             block_mask=None, grad_dtype=None, path: int = PATH_AUTO, workspace=None):
+             block_mask=None, grad_dtype=None, path: int = PATH_AUTO, workspace=None,
+             deterministic: bool = False):
     """dQ, dK, dV of sum(O * dO). grad_dtype defaults to float32 (the tensor
-    cores accumulate in fp32; a bf16 gradient adds its own rounding)."""
+    cores accumulate in fp32; a bf16 gradient adds its own rounding).
+    deterministic: run-to-run identical dQ (fa_bwd_deterministic)."""
     import torch
     B, Hq, Hkv, N, d = _dims(q, k)
     if scale is None:
@@ -226,11 +234,11 @@ def backward(q, k, v, o, do, lse, scale: Optional[float] = None, causal: bool = 
     dv = torch.empty(v.shape, dtype=gdt, device=q.device)
     nbytes = fa_bwd_workspace_size(B, Hq, N, d)
     ws = new_workspace(nbytes, q.device) if workspace is None else workspace
-    s = fa_bwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
-                  _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _ptr(block_mask),
-                  _dtype_code(q.dtype), _dtype_code(gdt), _ptr(ws), ws.numel(), _stream(),
-                  int(path))
-    _check(s, "fa_bwd")
+    fn = fa_bwd_deterministic if deterministic else fa_bwd_ex
+    s = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+           _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _ptr(block_mask),
+           _dtype_code(q.dtype), _dtype_code(gdt), _ptr(ws), ws.numel(), _stream(), int(path))
+    _check(s, "fa_bwd_deterministic" if deterministic else "fa_bwd")
     return dq, dk, dv
 
 

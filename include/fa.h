@@ -157,6 +157,23 @@ fa_status fa_bwd_finalize(const void* Q, const void* K, const void* V, const voi
                           void* workspace, size_t workspace_bytes, void* stream, int path);
 
 /*
+ * fa_bwd with run-to-run identical gradients. fa_bwd adds the dQ partials of
+ * different key tiles with fp32 reduce-adds whose order depends on
+ * scheduling, so its dQ can differ in the last bits between runs (dK, dV
+ * and the forward are identical run to run). Here the main kernel skips dQ
+ * and a second kernel computes it per 128-row query tile, summing the key
+ * tiles in a fixed order in TMEM: 3 more matrix products per (query tile,
+ * key tile) pair (S, dP, dQ), so about 60 % more backward work. Arguments,
+ * workspace and errors as fa_bwd_ex (path: FA_PATH_*; the CUDA-core kernels
+ * are deterministic already). Not for variable-length batches.
+ */
+fa_status fa_bwd_deterministic(const void* Q, const void* K, const void* V, const void* O,
+                               const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                               int B, int Hq, int Hkv, int N, int d, float scale, int causal,
+                               const uint8_t* block_mask, int dtype, int grad_dtype,
+                               void* workspace, size_t workspace_bytes, void* stream, int path);
+
+/*
  * Variable-length (padding-free) batches. The glossary page ("Sequence Length
  * Flexibility") names arbitrary sequence lengths without padding; these entry
  * points take B sequences packed back to back:
