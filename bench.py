@@ -60,15 +60,17 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--deterministic", action="store_true",
+                    help="backward through fa_bwd_deterministic (run-to-run identical dQ)")
     return ap.parse_args()
 
 
-def workload_config(w: inputs.Workload, world: int) -> dict:
+def workload_config(w: inputs.Workload, world: int, deterministic: bool = False) -> dict:
     return {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} "
                         f"{'causal' if w.causal else 'non-causal'}"
                         f"{' block-sparse' if w.sparse else ''} bf16 fwd+bwd",
             "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
-            "block_sparse": w.sparse, "grad_dtype": "f32",
+            "block_sparse": w.sparse, "grad_dtype": "f32", "deterministic_dq": deterministic,
             "parallelism": f"replicas x{world} (independent batches)",
             "l2": "no flush: each of Q, K, V, dO is larger than L2 (126 MB)"
                   if w.B * w.Hq * w.N * w.d * 2 > 126e6 else "working set may fit L2"}
@@ -276,6 +278,15 @@ def run_ours(args):
               ("bwd_preprocess", lambda: fa.fa_bwd_preprocess(*bwd_args)),
               ("bwd_main", lambda: fa.fa_bwd_main(*bwd_args)),
               ("bwd_finalize", lambda: fa.fa_bwd_finalize(*bwd_args))]
+    if args.deterministic:
+        # one stage: preprocess, main kernel without dQ, per-query-tile dQ kernel
+        # (the empty stages make an ABI call that launches nothing, so the
+        # launch count stays exact)
+        noop = lambda: fa.fa_exp2_fma(0, 0, 0, 0)  # noqa: E731
+        stages = [("fwd", lambda: fa.fa_fwd_ex(*fwd_args)),
+                  ("bwd_preprocess", noop),
+                  ("bwd_main", lambda: fa.fa_bwd_deterministic(*bwd_args)),
+                  ("bwd_finalize", noop)]
     n_stage_ev = len(stages) + 1
 
     def step(evs=None):
@@ -375,7 +386,8 @@ def run_ours(args):
                           int(w.causal), P(mask), fa.FA_BF16, P(ws), sp)
             if s != fa.FA_OK:
                 raise RuntimeError(fa.status_string(s))
-            s = fa.fa_bwd(*bwd_args[:-1])
+            s = fa.fa_bwd_deterministic(*bwd_args) if args.deterministic else \
+                fa.fa_bwd(*bwd_args[:-1])
             if s != fa.FA_OK:
                 raise RuntimeError(fa.status_string(s))
             for dst, src in ((ho, o), (hl, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
@@ -408,7 +420,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) rounded to bf16)",
-            "config": workload_config(w, world),
+            "config": workload_config(w, world, args.deterministic),
             "stages_ms": per_stage, "per_direction": stage_frac, "roofline": roof,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
     if rank == 0:
