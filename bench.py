@@ -205,6 +205,27 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- multi-rank helpers
+
+def max_over_ranks(ms: float, device=None) -> float:
+    """The slowest rank's time (the whole job ends when it ends); ms itself
+    when not running under an initialised process group of more than one."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return ms
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(flops_per_rank_step: float, steps: int, world: int, ms: float) -> float:
+    """Whole-job throughput under weak scaling: every rank runs the same
+    per-rank workload (its own seeded batch), so the job does world times
+    the per-rank work in the slowest rank's time."""
+    return flops_per_rank_step * steps * world / (ms / 1e3) / 1e12
+
+
 # ---------------------------------------------------------------- our arm
 
 def measured_peaks():
@@ -328,11 +349,7 @@ def run_ours(args):
     torch.cuda.synchronize()
     barrier()
     clocks = sampler.stop()
-    ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     err = fa.device_error(ws)
     if err != fa.FA_OK:
         raise RuntimeError(f"device error word set during timing: {fa.status_string(err)}")
@@ -341,8 +358,7 @@ def run_ours(args):
                                        for i in range(args.steps))
                  for j, (name, _) in enumerate(stages)}
     fwd_fl, bwd_fl = step_flops(w, x["mask"])
-    total_fl = (fwd_fl + bwd_fl) * args.steps * world
-    value = total_fl / (ms / 1e3) / 1e12
+    value = job_tflops(fwd_fl + bwd_fl, args.steps, world, ms)
 
     # dominant kernel: the stage with the longest mean duration
     dom = max(per_stage, key=per_stage.get)
@@ -403,12 +419,8 @@ def run_ours(args):
         b_.record(stream)
         torch.cuda.synchronize()
         barrier()
-        ems = a.elapsed_time(b_)
-        if world > 1:
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
-        e2e = {"value": (fwd_fl + bwd_fl) * args.e2e_steps * world / (ems / 1e3) / 1e12,
+        ems = max_over_ranks(a.elapsed_time(b_), dev)
+        e2e = {"value": job_tflops(fwd_fl + bwd_fl, args.e2e_steps, world, ems),
                "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                "steps": args.e2e_steps}
 
