@@ -49,6 +49,8 @@ void fill_common(Problem& p, int B, int Hq, int Hkv, int N, int d, float scale, 
   p.d = d;
   p.scale = scale;
   p.causal = causal;
+  p.wl = -1;
+  p.wr = causal ? 0 : -1;
   p.mask = mask;
   p.nb = (N + 127) / 128;
   p.Npad = p.nb * 128;
@@ -97,10 +99,15 @@ size_t fa_bwd_workspace_size(int B, int Hq, int N, int d) {
   return kErrBlock + 2 * vec + acc;
 }
 
-fa_status fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+}  // extern "C"
+
+namespace fa {
+namespace {
+
+fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                     int Hq, int Hkv, int N, int d, float scale, int causal,
                     const uint8_t* block_mask, int dtype, void* workspace, void* stream,
-                    int path) {
+                    int path, int wl = -1, int wr = -2) {
   t_launches = 0;
   fa_status s = check_dims(B, Hq, Hkv, N, d, scale, causal, dtype);
   if (s != FA_OK) return s;
@@ -119,10 +126,40 @@ fa_status fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float*
   p.Oout = O;
   p.LSEout = LSE;
   p.err = static_cast<unsigned*>(workspace);
+  const bool windowed = wl >= 0 || wr >= -1;
+  if (windowed) {
+    // a window runs on the tensor-core kernels only
+    p.wl = wl;
+    p.wr = causal ? 0 : wr;
+    if (path == FA_PATH_SIMT) return FA_ERR_UNSUPPORTED;
+    path = FA_PATH_TC;
+  }
   const bool tc_ok = sm100_fwd_supported(p);
   if (path == FA_PATH_TC && !tc_ok) return FA_ERR_UNSUPPORTED;
   const bool use_tc = (path == FA_PATH_TC) || (path == FA_PATH_AUTO && tc_ok);
   return from_cuda(use_tc ? sm100_fwd(p) : simt_fwd(p));
+}
+
+}  // namespace
+}  // namespace fa
+
+extern "C" {
+
+fa_status fa_fwd_ex(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                    int Hq, int Hkv, int N, int d, float scale, int causal,
+                    const uint8_t* block_mask, int dtype, void* workspace, void* stream,
+                    int path) {
+  return fwd_impl(Q, K, V, O, LSE, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype, workspace,
+                  stream, path);
+}
+
+fa_status fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                        int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
+                        int window_right, const uint8_t* block_mask, int dtype, void* workspace,
+                        void* stream) {
+  if (window_left < -1 || window_right < -1) return FA_ERR_INVALID_ARG;
+  return fwd_impl(Q, K, V, O, LSE, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype, workspace,
+                  stream, FA_PATH_AUTO, window_left, window_right);
 }
 
 fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
@@ -144,7 +181,7 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
                    int N, int d, float scale, int causal, const uint8_t* block_mask, int dtype,
                    int grad_dtype, void* workspace, size_t workspace_bytes, void* stream,
                    int path, int stages, const int* cu = nullptr, int total = 0,
-                   int deterministic = 0) {
+                   int deterministic = 0, int wl = -1, int wr = -2) {
   t_launches = 0;
   fa_status s = check_dims(B, Hq, Hkv, N, d, scale, causal, dtype);
   if (s != FA_OK) return s;
@@ -165,6 +202,13 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   fill_common(p, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype, stream);
   p.cu = cu;
   p.total = total;
+  if (wl >= 0 || wr >= -1) {
+    // a window runs on the tensor-core kernels only
+    p.wl = wl;
+    p.wr = causal ? 0 : wr;
+    if (path == FA_PATH_SIMT) return FA_ERR_UNSUPPORTED;
+    path = FA_PATH_TC;
+  }
   p.Q = Q;
   p.K = K;
   p.V = V;
@@ -254,6 +298,17 @@ fa_status fa_bwd(const void* Q, const void* K, const void* V, const void* O, con
 FA_STAGE_ENTRY(fa_bwd_preprocess, kPre)
 FA_STAGE_ENTRY(fa_bwd_main, kMain)
 FA_STAGE_ENTRY(fa_bwd_finalize, kFinal)
+
+fa_status fa_bwd_window(const void* Q, const void* K, const void* V, const void* O,
+                        const void* dO, const float* LSE, void* dQ, void* dK, void* dV, int B,
+                        int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
+                        int window_right, const uint8_t* block_mask, int dtype, int grad_dtype,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  if (window_left < -1 || window_right < -1) return FA_ERR_INVALID_ARG;
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, Hq, Hkv, N, d, scale, causal, block_mask,
+                  dtype, grad_dtype, workspace, workspace_bytes, stream, FA_PATH_AUTO, kAll,
+                  nullptr, 0, 0, window_left, window_right);
+}
 
 fa_status fa_bwd_deterministic(const void* Q, const void* K, const void* V, const void* O,
                                const void* dO, const float* LSE, void* dQ, void* dK, void* dV,

@@ -25,6 +25,9 @@ struct Problem {
   int B = 0, Hq = 0, Hkv = 0, N = 0, d = 0;
   float scale = 1.f;
   int causal = 0;
+  // sliding window: visible keys j of query i satisfy i - wl <= j <= i + wr
+  // (-1: unbounded); the launchers apply the causal flag as wr = 0 on top
+  int wl = -1, wr = -1;
   const uint8_t* mask = nullptr;  // [nb * nb] or null
   int nb = 0;                     // ceil(N / 128)
   int dtype = 0;                  // 0 f32, 1 bf16

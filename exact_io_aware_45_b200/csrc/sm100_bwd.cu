@@ -108,6 +108,7 @@ struct BwdParams {
   const uint8_t* mask;
   unsigned* err;
   int N, Npad, Hq, Hkv, nb, causal, grad_bf16, BHk;
+  int wl, wr;                  // visible keys: row - wl <= key <= row + wr (-1: unbounded)
   float c;                     // scale * log2(e)
   float scale;
   const int* cu;               // variable-length batch: sequence offsets [B+1], or null
@@ -181,11 +182,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   if (warp == 3) {
     // Query tiles that can see this key tile, in increasing order.
     const int nqt = (N + MQ - 1) / MQ;
-    const int qt_lo = p.causal ? n0 / MQ : 0;
+    // first query tile whose last row reaches the window of this key tile
+    const int qt_lo = p.wr >= 0 ? max(0, (n0 - p.wr) / MQ) : 0;
     int count = 0;
     for (int t0 = qt_lo; t0 < nqt; t0 += 32) {
       const int qt = t0 + lane;
-      const bool vis = qt < nqt && (!p.mask || p.mask[(size_t)((qt * MQ) / 128) * p.nb + kb]);
+      const bool vis = qt < nqt && (!p.mask || p.mask[(size_t)((qt * MQ) / 128) * p.nb + kb]) &&
+                       win_any(qt * MQ, qt * MQ + MQ - 1, n0, n0 + kBN - 1, p.wl, p.wr);
       const unsigned bal = __ballot_sync(0xffffffffu, vis);
       if (vis) ctl.qtiles[count + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(qt);
       count += __popc(bal);
@@ -332,8 +335,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           mma_commit(&ctl.sp_full[1]);
         }
         for (int i = 0; ok && i < n_items; ++i) {
-          // d = 128: one signal per item (per-chunk signals measured slower)
-          if (!(ok = mbar_wait(&ctl.p_ready[1], i & 1, g))) break;
+          // d = 128: one signal per item (per-chunk signals measured slower),
+          // on p_ready[i & 1]. Two barriers by item parity: S(i+1) is ready
+          // while item i's softmax runs, so a fast warp may arrive for item
+          // i+1 before a slow one arrives for item i; on one barrier that
+          // arrival could complete item i's phase early. Item i+2 cannot
+          // start before item i's phase completes (S(i+2) waits for dQ(i)).
+          if (!(ok = mbar_wait(&ctl.p_ready[i & 1], (i >> 1) & 1, g))) break;
           tc_fence_after();
           issue_dv(i, 0);
           issue_dv(i, 1);
@@ -401,7 +409,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       if (!mbar_wait(&ctl.qdo_full[s], (i / C::kStages) & 1, g)) break;
       tc_fence_after();
       const int q0 = item_q0(i);
-      const bool need_mask = kv >= N || (p.causal && q0 < n0 + kBN);
+      const bool need_mask =
+          kv >= N || win_cuts(q0, q0 + MQ - 1, n0, n0 + kBN - 1, p.wl, p.wr);
       const float* lse_s = vec + (s * 2 + 0) * MQ;
       const float* d_s = vec + (s * 2 + 1) * MQ;
       uint8_t* dsrow = base + C::kOffDS + (i & 1) * C::kDSBytes + r * 128;
@@ -422,8 +431,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           float p0 = ex2(fmaf(__uint_as_float(sv[e]), c, -la));
           float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), c, -lb));
           if (need_mask) {
-            if (kv >= N || (p.causal && qa_ < kv)) p0 = 0.f;
-            if (kv >= N || (p.causal && qa_ + 1 < kv)) p1 = 0.f;
+            if (kv >= N || !win_ok(qa_, kv, p.wl, p.wr)) p0 = 0.f;
+            if (kv >= N || !win_ok(qa_ + 1, kv, p.wl, p.wr)) p1 = 0.f;
           }
           const float g0 = p0 * (__uint_as_float(dp[e]) - da_);
           const float g1 = p1 * (__uint_as_float(dp[e + 1]) - db_);
@@ -442,14 +451,16 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           *reinterpret_cast<uint4*>(dsrow + blk * (kBN * 128) + ((c16 ^ (r & 7)) << 4)) = v;
         }
         // This chunk's P^T and dS^T are complete: for d = 64 the MMA warp
-        // may run the dV and dK steps over its query columns now; for d = 128
-        // it waits for the whole item (one signal after the last chunk).
+        // may run the dV and dK steps over its query columns now (p_ready[ch];
+        // item i+1's S is issued only after both steps of item i, so no warp
+        // runs an item ahead); for d = 128 it waits for the whole item (one
+        // signal after the last chunk, on p_ready[i & 1]).
         if (C::kSoftWarps == 8 || ch == kChunks - 1) {
           tmem_st_wait();
           fence_async_smem();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl.p_ready[ch]);
+          if (lane == 0) mbar_arrive(&ctl.p_ready[C::kDbl ? (i & 1) : ch]);
         }
       }
     }
@@ -602,6 +613,8 @@ cudaError_t launch(const Problem& pr) {
   kp.Hkv = pr.Hkv;
   kp.nb = pr.nb;
   kp.causal = pr.causal;
+  kp.wl = pr.wl;
+  kp.wr = pr.causal ? 0 : pr.wr;   // the causal flag is the window wr = 0
   kp.grad_bf16 = pr.grad_dtype == 1;
   kp.c = pr.scale * kLog2e;
   kp.scale = pr.scale;

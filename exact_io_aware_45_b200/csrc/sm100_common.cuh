@@ -144,6 +144,21 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// Visibility of key j to query i under a window (FlexAttention-style mask
+// modifier): i - wl <= j <= i + wr, a negative bound meaning unbounded. The
+// causal flag is the window wr = 0, wl unbounded.
+__device__ __forceinline__ bool win_ok(int i, int j, int wl, int wr) {
+  return (wr < 0 || j <= i + wr) && (wl < 0 || j >= i - wl);
+}
+// Some pair of query rows [r0, r1] and keys [c0, c1] is visible.
+__device__ __forceinline__ bool win_any(int r0, int r1, int c0, int c1, int wl, int wr) {
+  return (wr < 0 || c0 <= r1 + wr) && (wl < 0 || c1 >= r0 - wl);
+}
+// Some pair of query rows [r0, r1] and keys [c0, c1] is hidden by the window.
+__device__ __forceinline__ bool win_cuts(int r0, int r1, int c0, int c1, int wl, int wr) {
+  return (wr >= 0 && c1 > r0 + wr) || (wl >= 0 && c0 < r1 - wl);
+}
+
 // Maps a linear CTA index to (head, block) so that the blocks of `chunk`
 // heads are interleaved and, inside the chunk, issued from block 0 to
 // block nblk-1 (callers order their blocks by decreasing work). A wave then

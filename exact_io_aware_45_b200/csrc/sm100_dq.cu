@@ -69,6 +69,7 @@ struct DqParams {
   const uint8_t* mask;
   unsigned* err;
   int N, Npad, Hq, Hkv, nb, nqt, causal, BH, grad_bf16;
+  int wl, wr;                    // visible keys: row - wl <= key <= row + wr (-1: unbounded)
   float c;                       // scale * log2(e)
   float scale;
 };
@@ -119,11 +120,12 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
   }
   if (warp == 3) {
     // Key tiles this query tile sees, in increasing order.
-    const int kb_end = p.causal ? min(p.nb, qt + 1) : p.nb;
+    const int kb_end = p.wr >= 0 ? min(p.nb, (q0 + kBM - 1 + p.wr) / kBN + 1) : p.nb;
     int count = 0;
     for (int kb0 = 0; kb0 < kb_end; kb0 += 32) {
       const int kb = kb0 + lane;
-      const bool act = kb < kb_end && (!p.mask || p.mask[(size_t)qt * p.nb + kb]);
+      const bool act = kb < kb_end && (!p.mask || p.mask[(size_t)qt * p.nb + kb]) &&
+                       win_any(q0, q0 + kBM - 1, kb * kBN, kb * kBN + kBN - 1, p.wl, p.wr);
       const unsigned bal = __ballot_sync(0xffffffffu, act);
       if (act) ctl.tiles[count + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(kb);
       count += __popc(bal);
@@ -222,7 +224,8 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
       if (!mbar_wait(&ctl.sp_full, j & 1, g)) break;
       tc_fence_after();
       const int col0 = ctl.tiles[j] * kBN;
-      const bool need_mask = row >= N || col0 + kBN > N || (p.causal && col0 + kBN - 1 > q0);
+      const bool need_mask = row >= N || col0 + kBN > N ||
+                             win_cuts(q0, q0 + kBM - 1, col0, col0 + kBN - 1, p.wl, p.wr);
 #pragma unroll 1
       for (int ck = 0; ck < kBN / 32; ++ck) {
         uint32_t sv[32], dp[32];
@@ -234,8 +237,8 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
           float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), c, -lse2));
           if (need_mask) {
             const int k0 = col0 + ck * 32 + e;
-            if (row >= N || k0 >= N || (p.causal && k0 > row)) p0 = 0.f;
-            if (row >= N || k0 + 1 >= N || (p.causal && k0 + 1 > row)) p1 = 0.f;
+            if (row >= N || k0 >= N || !win_ok(row, k0, p.wl, p.wr)) p0 = 0.f;
+            if (row >= N || k0 + 1 >= N || !win_ok(row, k0 + 1, p.wl, p.wr)) p1 = 0.f;
           }
           pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dp[e]) - dd),
                                  p1 * (__uint_as_float(dp[e + 1]) - dd));
@@ -320,6 +323,8 @@ cudaError_t launch(const Problem& pr) {
   kp.nb = pr.nb;
   kp.nqt = pr.nb;   // 128-row query tiles
   kp.causal = pr.causal;
+  kp.wl = pr.wl;
+  kp.wr = pr.causal ? 0 : pr.wr;   // the causal flag is the window wr = 0
   kp.BH = (int)BHq;
   kp.grad_bf16 = pr.grad_dtype == 1;
   kp.c = pr.scale * kLog2e;

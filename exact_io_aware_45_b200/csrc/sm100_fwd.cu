@@ -93,6 +93,7 @@ struct FwdParams {
   const uint8_t* mask;
   unsigned* err;
   int N, Hq, Hkv, nb, nblk, causal, BH;
+  int wl, wr;                // visible keys: row - wl <= key <= row + wr (-1: unbounded)
   float c;                   // scale * log2(e)
   const int* cu;             // variable-length batch: sequence offsets [B+1], or null
   int total;                 // packed rows (variable-length batch)
@@ -185,15 +186,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   }
   if (warp == 3) {
     // Key tiles either query tile can see, in increasing order.
-    const int kb_end = p.causal ? min(nb, qb1 + 1) : nb;
+    const int kb_end = p.wr >= 0 ? min(nb, (qb1 * kBM + kBM - 1 + p.wr) / kBN + 1) : nb;
     int count = 0;
     for (int kb0 = 0; kb0 < kb_end; kb0 += 32) {
       const int kb = kb0 + lane;
       bool a0 = false, a1 = false;
       if (kb < kb_end) {
-        a0 = (!p.mask || p.mask[(size_t)qb0 * p.nb + kb]) && (!p.causal || kb <= qb0);
+        const int c0 = kb * kBN, c1 = c0 + kBN - 1;
+        a0 = (!p.mask || p.mask[(size_t)qb0 * p.nb + kb]) &&
+             win_any(qb0 * kBM, qb0 * kBM + kBM - 1, c0, c1, p.wl, p.wr);
         a1 = qb1 < nb && (!p.mask || p.mask[(size_t)qb1 * p.nb + kb]) &&
-             (!p.causal || kb <= qb1);
+             win_any(qb1 * kBM, qb1 * kBM + kBM - 1, c0, c1, p.wl, p.wr);
       }
       const bool act = a0 || a1;
       const unsigned bal = __ballot_sync(0xffffffffu, act);
@@ -336,12 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       tmem_ld128(sreg, sr);
       const int col0 = ctl.tiles[j] * kBN;
       const bool dead = (ctl.dead[j] >> t) & 1;
-      const bool need_mask = dead || col0 + kBN > N || (p.causal && col0 + kBN - 1 > tile_row0);
+      const bool need_mask = dead || col0 + kBN > N ||
+                             win_cuts(tile_row0, tile_row0 + kBM - 1, col0, col0 + kBN - 1, p.wl, p.wr);
       if (need_mask) {
 #pragma unroll
         for (int i = 0; i < 128; ++i) {
           const int col = col0 + i;
-          const bool bad = dead || col >= N || (p.causal && col > row);
+          const bool bad = dead || col >= N || !win_ok(row, col, p.wl, p.wr);
           if (bad) sr[i] = __float_as_uint(-INFINITY);
         }
       }
@@ -475,6 +479,8 @@ cudaError_t launch(const Problem& pr) {
   kp.nb = pr.nb;
   kp.nblk = (pr.N + 2 * kBM - 1) / (2 * kBM);
   kp.causal = pr.causal;
+  kp.wl = pr.wl;
+  kp.wr = pr.causal ? 0 : pr.wr;   // the causal flag is the window wr = 0
   kp.c = pr.scale * kLog2e;
   kp.cu = pr.cu;
   kp.total = pr.total;

@@ -28,7 +28,7 @@ EXPORTS = ("fa_status_string", "fa_version", "fa_fwd_workspace_size", "fa_bwd_wo
            "fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_preprocess", "fa_bwd_main",
            "fa_bwd_finalize", "fa_last_launch_count", "fa_get_device_error", "fa_exp2_fma",
            "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_size",
-           "fa_bwd_deterministic")
+           "fa_bwd_deterministic", "fa_fwd_window", "fa_bwd_window")
 
 _lib = None
 
@@ -80,6 +80,12 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd_varlen.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
                                     _I, _F, _I, _I, _I, _P, _S, _P]
         L.fa_bwd_varlen.restype = _I
+        L.fa_fwd_window.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _I, _I, _P,
+                                    _I, _P, _P]
+        L.fa_fwd_window.restype = _I
+        L.fa_bwd_window.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F,
+                                    _I, _I, _I, _P, _I, _I, _P, _S, _P]
+        L.fa_bwd_window.restype = _I
         L.fa_bwd_varlen_workspace_size.argtypes = [_I, _I, _I, _I, _I]
         L.fa_bwd_varlen_workspace_size.restype = _S
         _lib = L
@@ -146,6 +152,14 @@ def fa_exp2_fma(x_ptr: int, y_ptr: int, n: int, stream_ptr: int) -> int:
 
 def fa_bwd_deterministic(*args) -> int:
     return lib().fa_bwd_deterministic(*args)
+
+
+def fa_fwd_window(*args) -> int:
+    return lib().fa_fwd_window(*args)
+
+
+def fa_bwd_window(*args) -> int:
+    return lib().fa_bwd_window(*args)
 
 
 def fa_fwd_varlen(*args) -> int:
@@ -284,6 +298,44 @@ def backward_varlen(q, k, v, o, do, lse, cu_seqlens, max_seqlen: int,
                       d, float(scale), int(bool(causal)), _dtype_code(q.dtype), _dtype_code(gdt),
                       _ptr(ws), ws.numel(), _stream())
     _check(s, "fa_bwd_varlen")
+    return dq, dk, dv
+
+
+def forward_window(q, k, v, window_left: int, window_right: int, scale: Optional[float] = None,
+                   causal: bool = False, block_mask=None):
+    """O, LSE of sliding-window attention (fa_fwd_window); layouts as forward."""
+    import torch
+    B, Hq, Hkv, N, d = _dims(q, k)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    l = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    ws = new_workspace(fa_fwd_workspace_size(), q.device)
+    s = fa_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, float(scale),
+                      int(bool(causal)), int(window_left), int(window_right), _ptr(block_mask),
+                      _dtype_code(q.dtype), _ptr(ws), _stream())
+    _check(s, "fa_fwd_window")
+    return o, l
+
+
+def backward_window(q, k, v, o, do, lse, window_left: int, window_right: int,
+                    scale: Optional[float] = None, causal: bool = False, block_mask=None,
+                    grad_dtype=None):
+    """dQ, dK, dV of sliding-window attention (fa_bwd_window)."""
+    import torch
+    B, Hq, Hkv, N, d = _dims(q, k)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    gdt = torch.float32 if grad_dtype is None else grad_dtype
+    dq = torch.empty(q.shape, dtype=gdt, device=q.device)
+    dk = torch.empty(k.shape, dtype=gdt, device=q.device)
+    dv = torch.empty(v.shape, dtype=gdt, device=q.device)
+    ws = new_workspace(fa_bwd_workspace_size(B, Hq, N, d), q.device)
+    s = fa_bwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq),
+                      _ptr(dk), _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)),
+                      int(window_left), int(window_right), _ptr(block_mask), _dtype_code(q.dtype),
+                      _dtype_code(gdt), _ptr(ws), ws.numel(), _stream())
+    _check(s, "fa_bwd_window")
     return dq, dk, dv
 
 

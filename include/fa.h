@@ -157,6 +157,32 @@ fa_status fa_bwd_finalize(const void* Q, const void* K, const void* V, const voi
                           void* workspace, size_t workspace_bytes, void* stream, int path);
 
 /*
+ * Sliding-window (local) attention: a mask modifier on top of the causal flag
+ * and the block mask, in the spirit of the lesson's FlexAttention note (one
+ * tiled kernel, many masks; Researcher section, "Version lineage"). Key j is
+ * visible to query i iff
+ *   (window_left  < 0 or j >= i - window_left) and
+ *   (window_right < 0 or j <= i + window_right) and (causal == 0 or j <= i)
+ * and the block mask allows it; -1 means unbounded (the causal flag wins over
+ * window_right). Key tiles wholly outside the window are skipped, partly
+ * covered ones masked element by element. Same arguments, layouts and
+ * workspace rules as fa_fwd / fa_bwd otherwise; the backward must get the
+ * forward's window. Tensor-core kernels only (bf16, d in {64, 128},
+ * scale > 0): FA_ERR_UNSUPPORTED otherwise; FA_ERR_INVALID_ARG for a bound
+ * below -1.
+ */
+fa_status fa_fwd_window(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                        int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
+                        int window_right, const uint8_t* block_mask, int dtype, void* workspace,
+                        void* stream);
+
+fa_status fa_bwd_window(const void* Q, const void* K, const void* V, const void* O,
+                        const void* dO, const float* LSE, void* dQ, void* dK, void* dV, int B,
+                        int Hq, int Hkv, int N, int d, float scale, int causal, int window_left,
+                        int window_right, const uint8_t* block_mask, int dtype, int grad_dtype,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * fa_bwd with run-to-run identical gradients. fa_bwd adds the dQ partials of
  * different key tiles with fp32 reduce-adds whose order depends on
  * scheduling, so its dQ can differ in the last bits between runs (dK, dV

@@ -42,14 +42,21 @@ BLOCK = 128
 ROW_CHUNK = 512
 
 
-def allowed(rows: np.ndarray, N: int, causal: bool, block_mask) -> np.ndarray:
+def allowed(rows: np.ndarray, N: int, causal: bool, block_mask, window=None) -> np.ndarray:
     """Boolean [len(rows), N]: key j is visible to query i iff (not causal or
-    j <= i) and (no mask or mask[i // 128, j // 128])."""
+    j <= i) and (no mask or mask[i // 128, j // 128]) and, for a sliding
+    window (left, right) (a negative bound: unbounded), i - left <= j <= i + right."""
     rows = np.asarray(rows)
     cols = np.arange(N)
     ok = np.ones((rows.size, N), dtype=bool)
     if causal:
         ok &= cols[None, :] <= rows[:, None]
+    if window is not None:
+        left, right = window
+        if left >= 0:
+            ok &= cols[None, :] >= rows[:, None] - left
+        if right >= 0:
+            ok &= cols[None, :] <= rows[:, None] + right
     if block_mask is not None:
         ok &= block_mask[(rows // BLOCK)[:, None], (cols // BLOCK)[None, :]].astype(bool)
     return ok
@@ -75,7 +82,7 @@ def _kv_head(h: int, Hq: int, Hkv: int) -> int:
     return h // (Hq // Hkv)
 
 
-def forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows):
+def forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows, window=None):
     """O and LSE of query rows ``rows`` of head (b, h), in fp64."""
     Hq, Hkv, N = Q.shape[1], K.shape[1], K.shape[2]
     hk = _kv_head(h, Hq, Hkv)
@@ -87,14 +94,14 @@ def forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows):
     for c in range(0, rows.size, ROW_CHUNK):
         r = rows[c:c + ROW_CHUNK]
         S = scale * (Q[b, h, r].astype(np.float64) @ Kh.T)
-        S[~allowed(r, N, causal, block_mask)] = -np.inf
+        S[~allowed(r, N, causal, block_mask, window)] = -np.inf
         P, lse = softmax_rows(S)
         O[c:c + r.size] = P @ Vh
         L[c:c + r.size] = lse
     return O, L
 
 
-def forward(Q, K, V, scale, causal=False, block_mask=None):
+def forward(Q, K, V, scale, causal=False, block_mask=None, window=None):
     """O [B,Hq,N,d] and LSE [B,Hq,N] in fp64 for all heads."""
     B, Hq, N, d = Q.shape
     O = np.empty((B, Hq, N, d))
@@ -102,11 +109,13 @@ def forward(Q, K, V, scale, causal=False, block_mask=None):
     rows = np.arange(N)
     for b in range(B):
         for h in range(Hq):
-            O[b, h], L[b, h] = forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows)
+            O[b, h], L[b, h] = forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows,
+                                            window)
     return O, L
 
 
-def _head_grads(Qh, Kh, Vh, dOh, Oh, scale, causal, block_mask, rows, want_dq=True):
+def _head_grads(Qh, Kh, Vh, dOh, Oh, scale, causal, block_mask, rows, want_dq=True,
+                window=None):
     """Gradient pieces of one query head restricted to query rows ``rows``.
 
     Returns (dQ_rows or None, dK contribution [N,d], dV contribution [N,d]).
@@ -118,7 +127,7 @@ def _head_grads(Qh, Kh, Vh, dOh, Oh, scale, causal, block_mask, rows, want_dq=Tr
     for c in range(0, rows.size, ROW_CHUNK):
         r = rows[c:c + ROW_CHUNK]
         S = scale * (Qh[r] @ Kh.T)
-        S[~allowed(r, N, causal, block_mask)] = -np.inf
+        S[~allowed(r, N, causal, block_mask, window)] = -np.inf
         P, _ = softmax_rows(S)
         dP = dOh[r] @ Vh.T
         D = np.sum(dOh[r] * Oh[r], axis=1)
@@ -130,7 +139,7 @@ def _head_grads(Qh, Kh, Vh, dOh, Oh, scale, causal, block_mask, rows, want_dq=Tr
     return dQ, dK, dV
 
 
-def backward(Q, K, V, dO, scale, causal=False, block_mask=None, O=None):
+def backward(Q, K, V, dO, scale, causal=False, block_mask=None, O=None, window=None):
     """dQ [B,Hq,N,d], dK and dV [B,Hkv,N,d] in fp64.
 
     O is the oracle's own forward output (recomputed here when not given).
@@ -138,7 +147,7 @@ def backward(Q, K, V, dO, scale, causal=False, block_mask=None, O=None):
     B, Hq, N, d = Q.shape
     Hkv = K.shape[1]
     if O is None:
-        O, _ = forward(Q, K, V, scale, causal, block_mask)
+        O, _ = forward(Q, K, V, scale, causal, block_mask, window)
     dQ = np.zeros((B, Hq, N, d))
     dK = np.zeros((B, Hkv, N, d))
     dV = np.zeros((B, Hkv, N, d))
@@ -148,7 +157,8 @@ def backward(Q, K, V, dO, scale, causal=False, block_mask=None, O=None):
             hk = _kv_head(h, Hq, Hkv)
             dq, dk, dv = _head_grads(Q[b, h].astype(np.float64), K[b, hk].astype(np.float64),
                                      V[b, hk].astype(np.float64), dO[b, h].astype(np.float64),
-                                     O[b, h], scale, causal, block_mask, rows)
+                                     O[b, h], scale, causal, block_mask, rows,
+                                     window=window)
             dQ[b, h] = dq
             dK[b, hk] += dk
             dV[b, hk] += dv
