@@ -411,6 +411,9 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       const int q0 = item_q0(i);
       const bool need_mask =
           kv >= N || win_cuts(q0, q0 + MQ - 1, n0, n0 + kBN - 1, p.wl, p.wr);
+      // queries that see this thread's key: [qlo, qhi] (empty past N)
+      const int qlo = (p.wr >= 0) ? kv - p.wr : 0;
+      const int qhi = (kv >= N) ? -1 : ((p.wl >= 0) ? kv + p.wl : 0x7fffffff);
       const float* lse_s = vec + (s * 2 + 0) * MQ;
       const float* d_s = vec + (s * 2 + 1) * MQ;
       uint8_t* dsrow = base + C::kOffDS + (i & 1) * C::kDSBytes + r * 128;
@@ -431,8 +434,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           float p0 = ex2(fmaf(__uint_as_float(sv[e]), c, -la));
           float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), c, -lb));
           if (need_mask) {
-            if (kv >= N || !win_ok(qa_, kv, p.wl, p.wr)) p0 = 0.f;
-            if (kv >= N || !win_ok(qa_ + 1, kv, p.wl, p.wr)) p1 = 0.f;
+            if (qa_ < qlo || qa_ > qhi) p0 = 0.f;
+            if (qa_ + 1 < qlo || qa_ + 1 > qhi) p1 = 0.f;
           }
           const float g0 = p0 * (__uint_as_float(dp[e]) - da_);
           const float g1 = p1 * (__uint_as_float(dp[e + 1]) - db_);
@@ -613,8 +616,9 @@ cudaError_t launch(const Problem& pr) {
   kp.Hkv = pr.Hkv;
   kp.nb = pr.nb;
   kp.causal = pr.causal;
-  kp.wl = pr.wl;
-  kp.wr = pr.causal ? 0 : pr.wr;   // the causal flag is the window wr = 0
+  // a bound of N or more cuts nothing: unbounded (keeps row +- bound in int range)
+  kp.wl = (pr.wl >= pr.N) ? -1 : pr.wl;
+  kp.wr = pr.causal ? 0 : ((pr.wr >= pr.N) ? -1 : pr.wr);   // causal is the window wr = 0
   kp.grad_bf16 = pr.grad_dtype == 1;
   kp.c = pr.scale * kLog2e;
   kp.scale = pr.scale;

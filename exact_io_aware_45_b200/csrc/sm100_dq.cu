@@ -226,6 +226,9 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
       const int col0 = ctl.tiles[j] * kBN;
       const bool need_mask = row >= N || col0 + kBN > N ||
                              win_cuts(q0, q0 + kBM - 1, col0, col0 + kBN - 1, p.wl, p.wr);
+      // this row's visible keys: [klo, khi] (empty past N)
+      const int klo = (p.wl >= 0) ? row - p.wl : 0;
+      const int khi = (row >= N) ? -1 : min(N - 1, (p.wr >= 0) ? row + p.wr : N - 1);
 #pragma unroll 1
       for (int ck = 0; ck < kBN / 32; ++ck) {
         uint32_t sv[32], dp[32];
@@ -237,8 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
           float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), c, -lse2));
           if (need_mask) {
             const int k0 = col0 + ck * 32 + e;
-            if (row >= N || k0 >= N || !win_ok(row, k0, p.wl, p.wr)) p0 = 0.f;
-            if (row >= N || k0 + 1 >= N || !win_ok(row, k0 + 1, p.wl, p.wr)) p1 = 0.f;
+            if (k0 < klo || k0 > khi) p0 = 0.f;
+            if (k0 + 1 < klo || k0 + 1 > khi) p1 = 0.f;
           }
           pk[e >> 1] = pack_bf16(p0 * (__uint_as_float(dp[e]) - dd),
                                  p1 * (__uint_as_float(dp[e + 1]) - dd));
@@ -323,8 +326,9 @@ cudaError_t launch(const Problem& pr) {
   kp.nb = pr.nb;
   kp.nqt = pr.nb;   // 128-row query tiles
   kp.causal = pr.causal;
-  kp.wl = pr.wl;
-  kp.wr = pr.causal ? 0 : pr.wr;   // the causal flag is the window wr = 0
+  // a bound of N or more cuts nothing: unbounded (keeps row +- bound in int range)
+  kp.wl = (pr.wl >= pr.N) ? -1 : pr.wl;
+  kp.wr = pr.causal ? 0 : ((pr.wr >= pr.N) ? -1 : pr.wr);   // causal is the window wr = 0
   kp.BH = (int)BHq;
   kp.grad_bf16 = pr.grad_dtype == 1;
   kp.c = pr.scale * kLog2e;

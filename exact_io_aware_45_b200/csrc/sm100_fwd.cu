@@ -342,12 +342,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const bool need_mask = dead || col0 + kBN > N ||
                              win_cuts(tile_row0, tile_row0 + kBM - 1, col0, col0 + kBN - 1, p.wl, p.wr);
       if (need_mask) {
+        // this row's visible columns of the tile: [lo, hi] relative to col0
+        int lo = (p.wl >= 0) ? row - p.wl - col0 : 0;
+        int hi = min(N - 1, (p.wr >= 0) ? row + p.wr : N - 1) - col0;
+        if (dead) hi = lo - 1;
 #pragma unroll
-        for (int i = 0; i < 128; ++i) {
-          const int col = col0 + i;
-          const bool bad = dead || col >= N || !win_ok(row, col, p.wl, p.wr);
-          if (bad) sr[i] = __float_as_uint(-INFINITY);
-        }
+        for (int i = 0; i < 128; ++i)
+          if (i < lo || i > hi) sr[i] = __float_as_uint(-INFINITY);
       }
       // Row maximum: eight independent chains of three-input max.
       float m8[8];
@@ -479,8 +480,9 @@ cudaError_t launch(const Problem& pr) {
   kp.nb = pr.nb;
   kp.nblk = (pr.N + 2 * kBM - 1) / (2 * kBM);
   kp.causal = pr.causal;
-  kp.wl = pr.wl;
-  kp.wr = pr.causal ? 0 : pr.wr;   // the causal flag is the window wr = 0
+  // a bound of N or more cuts nothing: unbounded (keeps row +- bound in int range)
+  kp.wl = (pr.wl >= pr.N) ? -1 : pr.wl;
+  kp.wr = pr.causal ? 0 : ((pr.wr >= pr.N) ? -1 : pr.wr);   // causal is the window wr = 0
   kp.c = pr.scale * kLog2e;
   kp.cu = pr.cu;
   kp.total = pr.total;

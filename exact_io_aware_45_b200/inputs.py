@@ -218,3 +218,15 @@ def varlen_lengths(total_target: int, lo: int, hi: int, seed: int = 0):
 def varlen_allowed_count(lengths, causal: bool) -> int:
     """Score elements a variable-length batch computes (per head)."""
     return sum(allowed_count(n, causal, None) for n in lengths)
+
+
+def window_allowed_count(N: int, causal: bool, left: int, right: int) -> int:
+    """Score elements per head under a sliding window (key j visible to
+    query i iff i - left <= j <= i + right, -1 unbounded, and j <= i when
+    causal), without materialising the N x N pattern."""
+    i = np.arange(N, dtype=np.int64)
+    lo = np.zeros(N, dtype=np.int64) if left < 0 else np.maximum(i - left, 0)
+    hi = np.full(N, N - 1, dtype=np.int64) if right < 0 else np.minimum(i + right, N - 1)
+    if causal:
+        hi = np.minimum(hi, i)
+    return int(np.maximum(hi - lo + 1, 0).sum())
