@@ -60,17 +60,22 @@ def parse_args():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--window", type=int, default=-1,
+                    help="sliding window: each query sees at most this many earlier keys "
+                         "(fa_fwd_window / fa_bwd_window with left = W, on the causal workload)")
     ap.add_argument("--deterministic", action="store_true",
                     help="backward through fa_bwd_deterministic (run-to-run identical dQ)")
     return ap.parse_args()
 
 
-def workload_config(w: inputs.Workload, world: int, deterministic: bool = False) -> dict:
+def workload_config(w: inputs.Workload, world: int, deterministic: bool = False,
+                    window: int = -1) -> dict:
     return {"workload": f"{w.name}: B={w.B} Hq={w.Hq} Hkv={w.Hkv} N={w.N} d={w.d} "
                         f"{'causal' if w.causal else 'non-causal'}"
                         f"{' block-sparse' if w.sparse else ''} bf16 fwd+bwd",
             "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
             "block_sparse": w.sparse, "grad_dtype": "f32", "deterministic_dq": deterministic,
+            "window_left": window,
             "parallelism": f"replicas x{world} (independent batches)",
             "l2": "no flush: each of Q, K, V, dO is larger than L2 (126 MB)"
                   if w.B * w.Hq * w.N * w.d * 2 > 126e6 else "working set may fit L2"}
@@ -299,6 +304,18 @@ def run_ours(args):
               ("bwd_preprocess", lambda: fa.fa_bwd_preprocess(*bwd_args)),
               ("bwd_main", lambda: fa.fa_bwd_main(*bwd_args)),
               ("bwd_finalize", lambda: fa.fa_bwd_finalize(*bwd_args))]
+    if args.window >= 0:
+        # one stage each: fa_fwd_window, fa_bwd_window (preprocess, main, finalize)
+        noop = lambda: fa.fa_exp2_fma(0, 0, 0, 0)  # noqa: E731
+        wfa = (P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, float(w.scale), int(w.causal),
+               args.window, -1, P(mask), fa.FA_BF16, P(ws), sp)
+        wba = (P(q), P(k), P(v), P(o), P(do), P(lse), P(dq), P(dk), P(dv), B, Hq, Hkv, N, d,
+               float(w.scale), int(w.causal), args.window, -1, P(mask), fa.FA_BF16, fa.FA_F32,
+               P(ws), wsb, sp)
+        stages = [("fwd", lambda: fa.fa_fwd_window(*wfa)),
+                  ("bwd_preprocess", noop),
+                  ("bwd_main", lambda: fa.fa_bwd_window(*wba)),
+                  ("bwd_finalize", noop)]
     if args.deterministic:
         # one stage: preprocess, main kernel without dQ, per-query-tile dQ kernel
         # (the empty stages make an ABI call that launches nothing, so the
@@ -358,6 +375,9 @@ def run_ours(args):
                                        for i in range(args.steps))
                  for j, (name, _) in enumerate(stages)}
     fwd_fl, bwd_fl = step_flops(w, x["mask"])
+    if args.window >= 0:
+        allowed = inputs.window_allowed_count(N, w.causal, args.window, -1) * B * Hq
+        fwd_fl, bwd_fl = 4.0 * d * allowed, 10.0 * d * allowed
     value = job_tflops(fwd_fl + bwd_fl, args.steps, world, ms)
 
     # dominant kernel: the stage with the longest mean duration
@@ -398,12 +418,18 @@ def run_ours(args):
         def e2e_step():
             for dst, src in ((q, hq_), (k, hk_), (v, hv_), (do, hdo)):
                 dst.copy_(src, non_blocking=True)
-            s = fa.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, float(w.scale),
-                          int(w.causal), P(mask), fa.FA_BF16, P(ws), sp)
+            if args.window >= 0:
+                s = fa.fa_fwd_window(*wfa)
+            else:
+                s = fa.fa_fwd(P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, float(w.scale),
+                              int(w.causal), P(mask), fa.FA_BF16, P(ws), sp)
             if s != fa.FA_OK:
                 raise RuntimeError(fa.status_string(s))
-            s = fa.fa_bwd_deterministic(*bwd_args) if args.deterministic else \
-                fa.fa_bwd(*bwd_args[:-1])
+            if args.window >= 0:
+                s = fa.fa_bwd_window(*wba)
+            else:
+                s = fa.fa_bwd_deterministic(*bwd_args) if args.deterministic else \
+                    fa.fa_bwd(*bwd_args[:-1])
             if s != fa.FA_OK:
                 raise RuntimeError(fa.status_string(s))
             for dst, src in ((ho, o), (hl, lse), (hdq, dq), (hdk, dk), (hdv, dv)):
@@ -432,7 +458,7 @@ def run_ours(args):
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1) rounded to bf16)",
-            "config": workload_config(w, world, args.deterministic),
+            "config": workload_config(w, world, args.deterministic, args.window),
             "stages_ms": per_stage, "per_direction": stage_frac, "roofline": roof,
             "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
     if rank == 0:
