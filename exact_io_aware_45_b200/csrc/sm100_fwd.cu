@@ -5,7 +5,8 @@
 // keys and LSE = logsumexp(scale * Q K^T) (FlashAttention lesson, Researcher
 // section "The problem being solved"), never writing S or P to HBM (paper
 // summary, "Core Idea" items 1, 2 and 4). Each CTA owns two 128-row query tiles
-// of one (batch, head) and walks the key tiles both need; for each key tile j:
+// of one (batch, head) and walks the key tiles either needs (K and V are loaded
+// once for both); for each key tile j:
 //
 //   S_t = Q_t K_j^T             tcgen05.mma, A and B from shared memory, S in TMEM
 //   online softmax on S_t       one thread per row (tcgen05.ld 32x32b), base-2
@@ -31,6 +32,16 @@
 // tcgen05.mma operations issued by one thread execute in order, so the next
 // Q_t K^T that overwrites S_t cannot overtake the P_t V that reads it.
 //
+// A key tile one query tile sees nothing of (a block-mask cell that is off,
+// a window edge, the causal diagonal of the other tile) is either computed for
+// it fully masked, keeping the two tiles in lockstep (dense, causal and
+// variable-length launches, where there are at most one or two such tiles per
+// CTA), or skipped for it: no Q K^T, softmax or P V (kSkip: block-sparse masks
+// and windows with a left edge, where a random mask makes about 40% of the
+// halves dead). The skipping form counts barrier phases per query tile;
+// measured on B200 it is 4-12% slower than the lockstep form where nearly
+// every tile is seen by both query tiles, hence the two forms.
+//
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
 // TMEM allocator, warp 3 builds the key-tile list, warps 4-7 softmax of query
 // tile 0, warps 8-11 softmax of query tile 1.
@@ -51,7 +62,7 @@ constexpr int kThreads = 384;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kTau = 8.0f;       // reference-max slack, log2 units
-constexpr int kChunk = 16;         // heads interleaved in launch order
+constexpr int kMaxChunk = 16;      // most heads interleaved in launch order
 
 template <int D>
 struct Cfg {
@@ -78,12 +89,15 @@ struct alignas(16) Ctl {
   uint64_t q_full;
   uint64_t k_full[4], v_full[4], kv_empty[4];
   uint64_t s_full[2], p_half[2], p_full[2];
+  uint64_t o_ready[2];       // query tile t's last P V has completed (skipping form)
   uint64_t o_done;
   uint32_t tmem_base;
   int abort;
   int ntiles;
+  int nlive[2];                  // key tiles query tile t sees (skipping form)
   uint16_t tiles[kMaxTiles];
-  uint8_t dead[kMaxTiles];   // bit t: query tile t sees nothing of this key tile
+  uint8_t dead[kMaxTiles];       // bit t: query tile t sees nothing of this key tile
+  uint16_t seen[kMaxTiles][2];   // [n][t]: n-th key tile query tile t sees (skipping form)
 };
 
 struct FwdParams {
@@ -97,6 +111,7 @@ struct FwdParams {
   float c;                   // scale * log2(e)
   const int* cu;             // variable-length batch: sequence offsets [B+1], or null
   int total;                 // packed rows (variable-length batch)
+  int chunk;                 // heads interleaved in launch order
 };
 
 // 32 pairs of scores -> p = 2^(s*c - mu) packed to bf16 pairs, with the
@@ -127,7 +142,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int D, bool kVarlen>
+template <int D, bool kVarlen, bool kSkip>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -136,10 +151,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   const uint32_t tile_addr = (raw_addr + sizeof(Ctl) + 1023u) & ~1023u;
   uint8_t* tiles_base = smem_raw + (tile_addr - raw_addr);
 
-  // Heads are taken kChunk at a time (their K/V stay in L2 during a wave);
+  // Heads are taken p.chunk at a time (their K/V stay in L2 during a wave);
   // inside a chunk the query blocks with the longest causal rows start first.
   int bh, rblk;
-  chunked_order(blockIdx.x, p.nblk, p.BH, kChunk, bh, rblk);
+  chunked_order(blockIdx.x, p.nblk, p.BH, p.chunk, bh, rblk);
   // A launch whose error word is already set (an earlier wait ran out and
   // nobody has read the word yet) does no work: its inputs may be invalid.
   if (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) return;
@@ -175,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       mbar_init(&ctl.s_full[t], 1);
       mbar_init(&ctl.p_half[t], 4);
       mbar_init(&ctl.p_full[t], 4);
+      mbar_init(&ctl.o_ready[t], 1);
     }
     mbar_init(&ctl.o_done, 1);
     ctl.abort = 0;
@@ -187,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   if (warp == 3) {
     // Key tiles either query tile can see, in increasing order.
     const int kb_end = p.wr >= 0 ? min(nb, (qb1 * kBM + kBM - 1 + p.wr) / kBN + 1) : nb;
-    int count = 0;
+    int count = 0, live0 = 0, live1 = 0;
     for (int kb0 = 0; kb0 < kb_end; kb0 += 32) {
       const int kb = kb0 + lane;
       bool a0 = false, a1 = false;
@@ -205,9 +221,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         ctl.tiles[pos] = static_cast<uint16_t>(kb);
         ctl.dead[pos] = static_cast<uint8_t>((a0 ? 0 : 1) | (a1 ? 0 : 2));
       }
+      if constexpr (kSkip) {
+        // and each query tile's own list
+        const unsigned below = (1u << lane) - 1u;
+        const unsigned bal0 = __ballot_sync(0xffffffffu, a0);
+        const unsigned bal1 = __ballot_sync(0xffffffffu, a1);
+        if (a0) ctl.seen[live0 + __popc(bal0 & below)][0] = static_cast<uint16_t>(kb);
+        if (a1) ctl.seen[live1 + __popc(bal1 & below)][1] = static_cast<uint16_t>(kb);
+        live0 += __popc(bal0);
+        live1 += __popc(bal1);
+      }
       count += __popc(bal);
     }
-    if (lane == 0) ctl.ntiles = count;
+    if (lane == 0) {
+      ctl.ntiles = count;
+      ctl.nlive[0] = live0;
+      ctl.nlive[1] = live1;
+    }
   }
   tc_fence_before();
   __syncthreads();
@@ -279,42 +309,109 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                  sdesc_sw128(vt + kk * 16 * 128, C::kBlockBytes, 1024), idO, (acc || kk > 0));
         }
       };
-      bool ok = mbar_wait(&ctl.q_full, 0, g) && mbar_wait(&ctl.k_full[0], 0, g);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0, 0);
-        mma_commit(&ctl.s_full[0]);
-        issue_s(1, 0);
-        mma_commit(&ctl.s_full[1]);
-      }
-      for (int j = 0; ok && j < T; ++j) {
-        const int s = j % C::kStages;
-        const uint32_t ph = (j / C::kStages) & 1;
-        if (!(ok = mbar_wait(&ctl.v_full[s], ph, g) && mbar_wait(&ctl.p_half[0], j & 1, g)))
-          break;
-        tc_fence_after();
-        issue_pv(0, s, j > 0, 0);
-        if (!(ok = mbar_wait(&ctl.p_full[0], j & 1, g))) break;
-        tc_fence_after();
-        issue_pv(0, s, j > 0, 1);
-        const bool more = j + 1 < T;
-        const int s2 = (j + 1) % C::kStages;
-        if (more) {
-          if (!(ok = mbar_wait(&ctl.k_full[s2], ((j + 1) / C::kStages) & 1, g))) break;
+      if constexpr (kSkip) {
+        // A query tile skips the key tiles it sees nothing of (block mask,
+        // causal diagonal, window edge): no Q K^T, softmax or P V for it there.
+        // n0, n1 count the tiles each query tile has been through; its barriers
+        // (s_full, p_half, p_full) complete once per such tile. The live bits
+        // of a tile (bit t: query tile t sees it) are read one tile ahead, so
+        // no shared-memory load sits between a signal and the next issue.
+        const int nl0 = ctl.nlive[0], nl1 = ctl.nlive[1];
+        int n0 = 0, n1 = 0;
+        int live_next = T > 0 ? (~ctl.dead[0] & 3) : 0;
+        bool ok = mbar_wait(&ctl.q_full, 0, g) && mbar_wait(&ctl.k_full[0], 0, g);
+        if (ok) {
           tc_fence_after();
-          issue_s(0, s2);
-          mma_commit(&ctl.s_full[0]);
+          if (live_next & 1) {
+            issue_s(0, 0);
+            mma_commit(&ctl.s_full[0]);
+          }
+          if (live_next & 2) {
+            issue_s(1, 0);
+            mma_commit(&ctl.s_full[1]);
+          }
         }
-        if (!(ok = mbar_wait(&ctl.p_half[1], j & 1, g))) break;
-        tc_fence_after();
-        issue_pv(1, s, j > 0, 0);
-        if (!(ok = mbar_wait(&ctl.p_full[1], j & 1, g))) break;
-        tc_fence_after();
-        issue_pv(1, s, j > 0, 1);
-        mma_commit(&ctl.kv_empty[s]);
-        if (more) {
-          issue_s(1, s2);
+        for (int j = 0; ok && j < T; ++j) {
+          const int s = j % C::kStages;
+          const uint32_t ph = (j / C::kStages) & 1;
+          const bool more = j + 1 < T;
+          const int s2 = (j + 1) % C::kStages;
+          const int live_cur = live_next;
+          live_next = more ? (~ctl.dead[j + 1] & 3) : 0;
+          if (!(ok = mbar_wait(&ctl.v_full[s], ph, g))) break;
+          if (live_cur & 1) {
+            if (!(ok = mbar_wait(&ctl.p_half[0], n0 & 1, g))) break;
+            tc_fence_after();
+            issue_pv(0, s, n0 > 0, 0);
+            if (!(ok = mbar_wait(&ctl.p_full[0], n0 & 1, g))) break;
+            tc_fence_after();
+            issue_pv(0, s, n0 > 0, 1);
+            if (++n0 == nl0) mma_commit(&ctl.o_ready[0]);
+          }
+          if (more) {
+            if (!(ok = mbar_wait(&ctl.k_full[s2], ((j + 1) / C::kStages) & 1, g))) break;
+            tc_fence_after();
+            if (live_next & 1) {
+              issue_s(0, s2);
+              mma_commit(&ctl.s_full[0]);
+            }
+          }
+          if (live_cur & 2) {
+            if (!(ok = mbar_wait(&ctl.p_half[1], n1 & 1, g))) break;
+            tc_fence_after();
+            issue_pv(1, s, n1 > 0, 0);
+            if (!(ok = mbar_wait(&ctl.p_full[1], n1 & 1, g))) break;
+            tc_fence_after();
+            issue_pv(1, s, n1 > 0, 1);
+            if (++n1 == nl1) mma_commit(&ctl.o_ready[1]);
+          }
+          mma_commit(&ctl.kv_empty[s]);
+          if (more && (live_next & 2)) {
+            issue_s(1, s2);
+            mma_commit(&ctl.s_full[1]);
+          }
+        }
+        // Every query tile's epilogue gets its signal, also after an abort.
+        if (n0 != nl0 || nl0 == 0) mma_commit(&ctl.o_ready[0]);
+        if (n1 != nl1 || nl1 == 0) mma_commit(&ctl.o_ready[1]);
+      } else {
+        bool ok = mbar_wait(&ctl.q_full, 0, g) && mbar_wait(&ctl.k_full[0], 0, g);
+        if (ok) {
+          tc_fence_after();
+          issue_s(0, 0);
+          mma_commit(&ctl.s_full[0]);
+          issue_s(1, 0);
           mma_commit(&ctl.s_full[1]);
+        }
+        for (int j = 0; ok && j < T; ++j) {
+          const int s = j % C::kStages;
+          const uint32_t ph = (j / C::kStages) & 1;
+          if (!(ok = mbar_wait(&ctl.v_full[s], ph, g) && mbar_wait(&ctl.p_half[0], j & 1, g)))
+            break;
+          tc_fence_after();
+          issue_pv(0, s, j > 0, 0);
+          if (!(ok = mbar_wait(&ctl.p_full[0], j & 1, g))) break;
+          tc_fence_after();
+          issue_pv(0, s, j > 0, 1);
+          const bool more = j + 1 < T;
+          const int s2 = (j + 1) % C::kStages;
+          if (more) {
+            if (!(ok = mbar_wait(&ctl.k_full[s2], ((j + 1) / C::kStages) & 1, g))) break;
+            tc_fence_after();
+            issue_s(0, s2);
+            mma_commit(&ctl.s_full[0]);
+          }
+          if (!(ok = mbar_wait(&ctl.p_half[1], j & 1, g))) break;
+          tc_fence_after();
+          issue_pv(1, s, j > 0, 0);
+          if (!(ok = mbar_wait(&ctl.p_full[1], j & 1, g))) break;
+          tc_fence_after();
+          issue_pv(1, s, j > 0, 1);
+          mma_commit(&ctl.kv_empty[s]);
+          if (more) {
+            issue_s(1, s2);
+            mma_commit(&ctl.s_full[1]);
+          }
         }
       }
       mma_commit(&ctl.o_done);
@@ -332,13 +429,19 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const float c = p.c;
     const int tile_row0 = q0 + t * kBM;
     float m_ref = -INFINITY, l = 0.f;
-    for (int j = 0; j < T; ++j) {
-      if (!mbar_wait(&ctl.s_full[t], j & 1, g)) break;
+    // Lockstep form: every tile of the list, n = it. Skipping form: only the
+    // tiles this query tile sees, it = 2n + t walking entry [n][t] of its list.
+    constexpr int kStep = kSkip ? 2 : 1;
+    const int it_end = kSkip ? 2 * ctl.nlive[t] + t : T;
+    int it = kSkip ? t : 0;
+    for (; it < it_end; it += kStep) {
+      const int n = kSkip ? (it >> 1) : it;   // tiles of this query tile so far
+      if (!mbar_wait(&ctl.s_full[t], n & 1, g)) break;
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld128(sreg, sr);
-      const int col0 = ctl.tiles[j] * kBN;
-      const bool dead = (ctl.dead[j] >> t) & 1;
+      const int col0 = (kSkip ? (&ctl.seen[0][0])[it] : ctl.tiles[it]) * kBN;
+      const bool dead = !kSkip && ((ctl.dead[it] >> t) & 1);
       const bool need_mask = dead || col0 + kBN > N ||
                              win_cuts(tile_row0, tile_row0 + kBM - 1, col0, col0 + kBN - 1, p.wl, p.wr);
       if (need_mask) {
@@ -392,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           // The accumulator holds P V of earlier tiles (complete: the commit
           // that signalled S_t came after them); rescale it where the
           // reference moved, before any P V of this tile is issued.
-          if (__any_sync(0xffffffffu, grow && j > 0)) {
+          if (__any_sync(0xffffffffu, grow && n > 0)) {
 #pragma unroll
             for (int cc = 0; cc < D / 32; ++cc) {
               uint32_t o[32];
@@ -416,8 +519,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       if (lane == 0) mbar_arrive(&ctl.p_full[t]);
     }
     // ------------------------------------------------------------ epilogue
-    if (T > 0) {
-      mbar_wait(&ctl.o_done, 0, g);
+    // The accumulator holds something only if some P V ran into it.
+    bool have_o;
+    if constexpr (kSkip)
+      have_o = __any_sync(0xffffffffu, it > 1);
+    else
+      have_o = T > 0;
+    if (have_o) {
+      mbar_wait(kSkip ? &ctl.o_ready[t] : &ctl.o_done, 0, g);
       tc_fence_after();
     }
     const float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -430,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 #pragma unroll
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t o[32];
-      if (T > 0) {
+      if (have_o) {
         tmem_ld32(oreg + cc * 32, o);
       } else {
 #pragma unroll
@@ -489,20 +598,33 @@ cudaError_t launch(const Problem& pr) {
   const size_t smem = sizeof(Ctl) + 1024 + C::kOffEnd;
   static bool attr_set = false;
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(fwd_kernel<D, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(fwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
-    if (e != cudaSuccess) return e;
+    for (const void* f : {(const void*)fwd_kernel<D, false, false>,
+                          (const void*)fwd_kernel<D, false, true>,
+                          (const void*)fwd_kernel<D, true, false>}) {
+      const cudaError_t e =
+          cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
     attr_set = true;
   }
   kp.BH = (int)BHq;
+  // As many heads at a time as keep their K and V within about half of the
+  // 126 MB L2 (heads sharing a KV head count once): 16 for 4K-16K sequences
+  // at d = 128, 4 for 64K at d = 64. Random block masks read K/V tiles out
+  // of order, so a working set larger than L2 turns into DRAM re-reads.
+  const uint64_t kv_bytes = 2ull * pr.N * D * 2;      // K and V of one KV head, bf16
+  const uint64_t per_kv = std::max<uint64_t>(1, (64ull << 20) / kv_bytes);
+  kp.chunk = (int)std::min<uint64_t>(kMaxChunk, std::max<uint64_t>(1, per_kv) * (pr.Hq / pr.Hkv));
   dim3 grid((unsigned)(BHq * kp.nblk));
+  // Skip dead query-tile halves where they are common: block-sparse masks and
+  // windows with a left edge (variable-length batches take neither).
+  const bool skip = !pr.cu && (pr.mask != nullptr || kp.wl >= 0);
   if (pr.cu)
-    fwd_kernel<D, true><<<grid, kThreads, smem, pr.stream>>>(kp);
+    fwd_kernel<D, true, false><<<grid, kThreads, smem, pr.stream>>>(kp);
+  else if (skip)
+    fwd_kernel<D, false, true><<<grid, kThreads, smem, pr.stream>>>(kp);
   else
-    fwd_kernel<D, false><<<grid, kThreads, smem, pr.stream>>>(kp);
+    fwd_kernel<D, false, false><<<grid, kThreads, smem, pr.stream>>>(kp);
   count_launch();
   return cudaGetLastError();
 }

@@ -128,6 +128,41 @@ def test_empty_block_row():
         assert_close_bf16("dV", to_np(r["dv"]), dV)
 
 
+BLOCK_PATTERNS = {
+    # the second query tile of the pair sees nothing
+    "lower_off": [[1, 1], [0, 0]],
+    # the first query tile of the pair sees nothing
+    "upper_off": [[0, 0], [1, 1]],
+    # every key tile is seen by exactly one tile of the first pair; the second
+    # pair has one empty row and one row with a gap
+    "alternating": [[1, 0, 1, 0], [0, 1, 0, 1], [0, 0, 0, 0], [1, 1, 0, 1]],
+}
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("pattern", sorted(BLOCK_PATTERNS))
+def test_block_mask_patterns(pattern, d):
+    """Block masks under which a query tile sees only some, or none, of the key
+    tiles its partner tile sees; rows with nothing visible give O = 0 and
+    LSE = -inf, the rest match the oracle."""
+    mask = np.array(BLOCK_PATTERNS[pattern], dtype=np.uint8)
+    N = 128 * mask.shape[0]
+    x = inputs.random_case(1, 2, 1, N, d, seed=11 + d)
+    x["mask"] = mask
+    scale = 1.0 / np.sqrt(d)
+    r = _run(x, scale, False, fa.PATH_AUTO)
+    o, lse = to_np(r["o"]), to_np(r["lse"])
+    O, L = orc.forward(x["q"], x["k"], x["v"], scale, False, mask)
+    empty = np.repeat(mask.sum(axis=1) == 0, 128)
+    assert np.all(o[:, :, empty] == 0) and np.all(np.isneginf(lse[:, :, empty]))
+    assert_close_bf16("O", o, O)
+    assert lse_err(lse[:, :, ~empty], L[:, :, ~empty]) <= LSE_MAX_ABS
+    dQ, dK, dV = orc.backward(x["q"], x["k"], x["v"], x["do"], scale, False, mask, O=O)
+    assert_close_bf16("dQ", to_np(r["dq"]), dQ)
+    assert_close_bf16("dK", to_np(r["dk"]), dK)
+    assert_close_bf16("dV", to_np(r["dv"]), dV)
+
+
 def test_forward_deterministic_and_fully_written():
     """Outputs are poisoned with NaN first; two runs agree bit for bit."""
     import torch
