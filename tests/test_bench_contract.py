@@ -1,6 +1,6 @@
 """The JSON line of bench.py's reference arm, on CPU: the arm times the fp64
 oracle on host cores, so it runs here. Checks the keys and types of the line
-a driver reads (metric, value, unit, steps, config, cpu_baseline, e2e) and that
+a caller parses (metric, value, unit, steps, config, cpu_baseline, e2e) and that
 the arm's value is the oracle's FLOPs over its own time, and that ranks other
 than 0 print nothing."""
 import json
