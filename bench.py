@@ -19,6 +19,10 @@ synchronisation on both sides and its duration is the maximum over ranks.
 ``--impl reference`` times the fp64 CPU oracle instead (the only other
 implementation of this computation here), on the same workload, metric and
 unit, one bounded sample (one batch-head, forward + backward) per step.
+
+``--workload fp32_n512_d32`` (one head, N = 512, d = 32, fp32, the lesson's
+NumPy example shape) has no backward: a step is one fp32 forward on the CUDA
+cores, L2 is flushed before each timed launch and only the launches are timed.
 """
 from __future__ import annotations
 
@@ -55,8 +59,7 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama7b_causal",
-                    choices=[k for k, w in inputs.WORKLOADS.items() if w.backward] +
-                    [VARLEN_NAME])
+                    choices=list(inputs.WORKLOADS) + [VARLEN_NAME])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -81,6 +84,14 @@ def workload_config(w: inputs.Workload, world: int, deterministic: bool = False,
                   if w.B * w.Hq * w.N * w.d * 2 > 126e6 else "working set may fit L2"}
 
 
+def forward_only_config(w: inputs.Workload, world: int) -> dict:
+    return {"workload": f"{w.name}: B={w.B} H={w.Hq} N={w.N} d={w.d} "
+                        f"{'causal' if w.causal else 'non-causal'} {w.dtype} forward",
+            "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
+            "block_sparse": w.sparse, "parallelism": f"replicas x{world} (independent batches)",
+            "l2": "flushed before every timed launch (a 256 MB write; inputs are 64 KB each)"}
+
+
 def step_flops(w: inputs.Workload, mask) -> tuple[float, float]:
     fwd = inputs.flops(w, mask=mask, backward=False)
     bwd = inputs.flops(w, mask=mask, backward=True)
@@ -99,31 +110,37 @@ def oracle_threads() -> int:
 
 
 def oracle_sample(w: inputs.Workload, x: dict, b: int, h: int):
-    """Runs the oracle forward + backward of one (batch, query head) and
-    returns (seconds, algorithmic FLOPs of that sample)."""
+    """Runs the oracle forward + backward (forward only for a workload
+    without a backward) of one (batch, query head) and returns (seconds,
+    algorithmic FLOPs of that sample)."""
     from oracle import attention as orc
     hk = h // w.group
     q = x["q"][b:b + 1, h:h + 1]
     k = x["k"][b:b + 1, hk:hk + 1]
     v = x["v"][b:b + 1, hk:hk + 1]
-    do = x["do"][b:b + 1, h:h + 1]
     t0 = time.perf_counter()
     O, _ = orc.forward(q, k, v, w.scale, w.causal, x["mask"])
-    orc.backward(q, k, v, do, w.scale, w.causal, x["mask"], O=O)
+    if w.backward:
+        do = x["do"][b:b + 1, h:h + 1]
+        orc.backward(q, k, v, do, w.scale, w.causal, x["mask"], O=O)
     dt = time.perf_counter() - t0
-    per = 14.0 * w.d * inputs.allowed_count(w.N, w.causal, x["mask"])
+    per = (14.0 if w.backward else 4.0) * w.d * inputs.allowed_count(w.N, w.causal, x["mask"])
     return dt, per
 
 
 def cpu_baseline(w, x, budget_s=20.0) -> dict:
     secs, fl, n = 0.0, 0.0, 0
-    while n == 0 or (secs < budget_s * 0.5 and n < 4):
+    # at least one unit; several while they are short (a forward-only unit of
+    # the fp32 workload takes milliseconds, so it is repeated)
+    cap = 4 if w.backward else 1000
+    while n == 0 or (secs < budget_s * 0.5 and n < cap):
         dt, f = oracle_sample(w, x, n % w.B, (n * 7) % w.Hq)
         secs += dt
         fl += f
         n += 1
+    what = "forward+backward" if w.backward else "forward"
     return {"value": fl / secs / 1e12, "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
-            "sample": f"{n} of {w.B * w.Hq} (batch, head) units, forward+backward in fp64 "
+            "sample": f"{n} (batch, head) units of {w.B * w.Hq}, {what} in fp64 "
                       f"NumPy ({secs:.1f} s)"}
 
 
@@ -146,10 +163,11 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * total / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": workload_config(w, world),
+            "config": workload_config(w, world) if w.backward else forward_only_config(w, world),
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": oracle_threads(),
                              "kind": "oracle",
-                             "sample": "one (batch, head) unit per step, forward+backward "
+                             "sample": "one (batch, head) unit per step, "
+                                       f"{'forward+backward' if w.backward else 'forward'} "
                                        "in fp64 NumPy"},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
@@ -468,6 +486,133 @@ def run_ours(args):
     return 0
 
 
+# ---------------------------------------------------------------- fp32 forward-only workload
+
+# fp32 FMA throughput: 148 SMs x 128 fp32 lanes x 2 FLOP per FMA at the 1,965 MHz maximum SM clock
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+
+
+def run_forward_only(args):
+    """One step = one fp32 forward (fa_fwd, CUDA-core kernel) of a workload
+    without a backward pass. Its inputs are far smaller than L2, so a 256 MB
+    buffer is written before every timed launch and only the launches are
+    timed (CUDA events around each); the step time is their sum."""
+    import torch
+    import torch.distributed as dist
+    from exact_io_aware_45_b200 import fa
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    fa.lib()
+
+    w = inputs.WORKLOADS[args.workload]
+    x = inputs.make_inputs(w, seed=rank)
+    q, k, v = (torch.from_numpy(x[n]).to(dev).contiguous() for n in ("q", "k", "v"))
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, N), dtype=torch.float32, device=dev)
+    ws = fa.new_workspace(fa.fa_fwd_workspace_size(), dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+    P = lambda t: t.data_ptr()  # noqa: E731
+    fargs = (P(q), P(k), P(v), P(o), P(lse), B, Hq, Hkv, N, d, float(w.scale), int(w.causal), 0,
+             fa.FA_F32, P(ws), sp)
+
+    def fwd():
+        s = fa.fa_fwd(*fargs)
+        if s != fa.FA_OK:
+            raise RuntimeError(f"fa_fwd: {fa.status_string(s)}")
+        return fa.fa_last_launch_count()
+
+    def barrier():
+        if world > 1:
+            dist.barrier(device_ids=[local])
+
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize()
+    if fa.device_error(ws) != fa.FA_OK:
+        raise RuntimeError("device error word set during warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    sampler = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    launches = 0
+    for i in range(args.steps):
+        flush.fill_(i & 255)
+        ev[i][0].record(stream)
+        launches += fwd()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in ev), dev)
+    if fa.device_error(ws) != fa.FA_OK:
+        raise RuntimeError("device error word set during timing")
+    fl = inputs.flops(w, mask=None, backward=False)
+    value = job_tflops(fl, args.steps, world, ms)
+    ach = fl / (ms / args.steps / 1e3) / 1e12
+    roof = {"bound": "alu", "kernel": "fwd (fp32 CUDA cores)", "achieved": ach,
+            "peak": FP32_FMA_PEAK_TFLOPS, "unit": "TFLOP/s", "frac": ach / FP32_FMA_PEAK_TFLOPS,
+            "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1,965 MHz",
+            "traffic": None}
+
+    e2e = None
+    if args.e2e_steps > 0:
+        hq_, hk_, hv_ = (torch.from_numpy(x[n]).pin_memory() for n in ("q", "k", "v"))
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hl = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in (hq_, hk_, hv_))
+        d2h = ho.numel() * ho.element_size() + hl.numel() * hl.element_size()
+
+        def e2e_step():
+            for dst, src in ((q, hq_), (k, hk_), (v, hv_)):
+                dst.copy_(src, non_blocking=True)
+            fwd()
+            for dst, src in ((ho, o), (hl, lse)):
+                dst.copy_(src, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier()
+        a, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        b_.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        ems = max_over_ranks(a.elapsed_time(b_), dev)
+        e2e = {"value": job_tflops(fl, args.e2e_steps, world, ems), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(w, x, budget_s=20.0)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+            "data": "synthetic (the lesson's NumPy draw: default_rng(0) normals, fp32)",
+            "config": forward_only_config(w, world), "roofline": roof, "cpu_baseline": cpu,
+            "e2e": e2e, "gpu_launches": launches, "clocks": clocks}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 # ---------------------------------------------------------------- variable-length batch
 
 VARLEN_NAME = "varlen_mix"
@@ -580,6 +725,8 @@ def main():
         return run_reference(args)
     if args.workload == VARLEN_NAME:
         return run_varlen(args)
+    if not inputs.WORKLOADS[args.workload].backward:
+        return run_forward_only(args)
     return run_ours(args)
 
 

@@ -84,3 +84,15 @@ def test_clock_sampler_without_nvidia_smi():
     import bench
     s = bench.ClockSampler(0)
     assert s.stop()["reasons"] == ["unavailable"]
+
+
+def test_reference_arm_forward_only_workload():
+    """The fp32 workload has no backward: the arm times the oracle forward and
+    counts 4 * d * N^2 FLOP per step."""
+    lines = _run(["--impl", "reference", "--workload", "fp32_n512_d32", "--steps", "2",
+                  "--warmup", "0"])
+    d = json.loads(lines[0])
+    assert d["config"]["workload"].startswith("fp32_n512_d32") and "forward" in d["config"]["workload"]
+    assert "forward+backward" not in d["cpu_baseline"]["sample"]
+    flops = 2 * 4 * 32 * 512 * 512
+    assert abs(d["value"] - flops / (2 * d["ms_per_step"] / 1e3) / 1e12) <= 1e-9 * d["value"]
