@@ -28,13 +28,15 @@ Everything is the plain definition: full rows of scores are formed (in row
 chunks only so that memory stays bounded; every row is complete before it is
 normalised). Disallowed pairs are set to -inf; a row with no allowed key gets
 O = 0, LSE = -inf and zero gradients. ``tiled_forward`` restates the pages'
-running-max / running-sum loop separately; it is used only to pin
-``forward`` against the pages' own worked example.
+online-softmax recurrence separately (as a fold of per-tile summaries); it is
+used only to pin ``forward`` against the pages' own worked example.
 
 Layouts: Q, dO, O [B, Hq, N, d]; K, V [B, Hkv, N, d]; LSE [B, Hq, N];
 block_mask uint8 [ceil(N/128), ceil(N/128)] shared by every (batch, head).
 """
 from __future__ import annotations
+
+import functools
 
 import numpy as np
 
@@ -213,44 +215,58 @@ def dkdv_rows(Q, K, V, dO, scale, causal, block_mask, b, hk, key_rows):
 
 
 def tiled_forward(Q2, K2, V2, scale, block, dtype=np.float64, trace=None):
-    """The pages' tiled loop for one head, restated (Developer section, "The
-    algorithm, in plain NumPy"; Researcher section, "Online softmax").
+    """The online-softmax recurrence for one head (lesson, Researcher section
+    "Online softmax", after Milakov and Gimelshein), written as a left fold of
+    per-tile summaries.
 
-    Key tiles of width ``block`` are visited in order while each query row
-    keeps m (running max), l (running sum of exponentials) and O (running
-    unnormalised output); when a tile raises m, l and O are multiplied by
-    exp(m_old - m_new) before the tile's own terms are added. Returns O / l.
-    All arithmetic is done in ``dtype``. If ``trace`` is a list, the number
-    of rows whose maximum grew is appended for each tile.
+    Key tile j (``block`` keys wide) is first summarised on its own as a
+    triple: its row maxima M_j, the row sums L_j of exp(S^(j) - M_j) and the
+    unnormalised partial output U_j = exp(S^(j) - M_j) V^(j). The running state
+    after tile j, (m^(j), l^(j), O^(j)), merges the state after tile j - 1 with
+    that triple: m^(j) = max(m^(j-1), M_j), and each side is carried onto the
+    new maximum by its own factor, exp(m^(j-1) - m^(j)) or exp(M_j - m^(j)),
+    before the two are added. Since rowsum(exp(S^(j) - m^(j))) equals
+    exp(M_j - m^(j)) L_j, this is the page's recurrence term for term; the
+    result is O^(T) / l^(T). All arithmetic is done in ``dtype``. If ``trace``
+    is a list, the number of rows whose running maximum grew is appended for
+    each tile.
     """
-    Q2 = Q2.astype(dtype)
-    K2 = K2.astype(dtype)
-    V2 = V2.astype(dtype)
-    n = Q2.shape[0]
-    m = np.full(n, -np.inf, dtype=dtype)
-    l = np.zeros(n, dtype=dtype)
-    acc = np.zeros((n, V2.shape[1]), dtype=dtype)
+    Q2, K2, V2 = (np.asarray(a_, dtype=dtype) for a_ in (Q2, K2, V2))
     sc = dtype(scale)
-    for j0 in range(0, K2.shape[0], block):
-        Sj = (Q2 @ K2[j0:j0 + block].T) * sc
-        m_new = np.maximum(m, Sj.max(axis=1))
+
+    def summary(j0):
+        S = (Q2 @ K2[j0:j0 + block].T) * sc
+        M = S.max(axis=1)
+        E = np.exp(S - M[:, None])
+        return M, E.sum(axis=1), E @ V2[j0:j0 + block]
+
+    def merge(state, tile):
+        m_prev, l_prev, O_prev = state
+        M, L, U = tile
+        m_next = np.maximum(m_prev, M)
         if trace is not None:
-            trace.append(int(np.count_nonzero(m_new > m)))
-        alpha = np.exp(m - m_new)
-        Pj = np.exp(Sj - m_new[:, None])
-        l = alpha * l + Pj.sum(axis=1)
-        acc = alpha[:, None] * acc + Pj @ V2[j0:j0 + block]
-        m = m_new
-    return acc / l[:, None]
+            trace.append(int(np.count_nonzero(m_next > m_prev)))
+        keep = np.exp(m_prev - m_next)     # 0 while nothing has been accumulated
+        bring = np.exp(M - m_next)
+        return m_next, keep * l_prev + bring * L, keep[:, None] * O_prev + bring[:, None] * U
+
+    rows = Q2.shape[0]
+    empty = (np.full(rows, -np.inf, dtype=dtype), np.zeros(rows, dtype=dtype),
+             np.zeros((rows, V2.shape[1]), dtype=dtype))
+    _, l_fin, O_fin = functools.reduce(merge, map(summary, range(0, K2.shape[0], block)), empty)
+    return O_fin / l_fin[:, None]
 
 
 def naive_forward_f32(Q2, K2, V2, scale):
-    """The pages' one-shot float32 reference for one head (the N x N score
-    matrix held in full, max-subtracted, exponentiated and normalised)."""
-    S = (Q2.astype(np.float32) @ K2.astype(np.float32).T) * np.float32(scale)
-    S = S - S.max(axis=1, keepdims=True)
-    P = np.exp(S)
-    return (P / P.sum(axis=1, keepdims=True)) @ V2.astype(np.float32)
+    """The one-shot float32 result for one head that the lesson checks its
+    loop against: the whole N x N score matrix is formed and every row is
+    normalised by its logsumexp (taken about the row maximum so that no
+    exponential overflows) before the product with V."""
+    f32 = np.float32
+    S = np.matmul(np.asarray(Q2, dtype=f32), np.asarray(K2, dtype=f32).T) * f32(scale)
+    top = S.max(axis=1, keepdims=True)
+    lse = top + np.log(np.exp(S - top).sum(axis=1, keepdims=True))
+    return np.exp(S - lse) @ np.asarray(V2, dtype=f32)
 
 
 # ---------------------------------------------------------------- variable-length batches
