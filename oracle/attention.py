@@ -44,24 +44,66 @@ BLOCK = 128
 ROW_CHUNK = 512
 
 
-def allowed(rows: np.ndarray, N: int, causal: bool, block_mask, window=None) -> np.ndarray:
-    """Boolean [len(rows), N]: key j is visible to query i iff (not causal or
-    j <= i) and (no mask or mask[i // 128, j // 128]) and, for a sliding
-    window (left, right) (a negative bound: unbounded), i - left <= j <= i + right."""
+def allowed(rows: np.ndarray, N: int, causal: bool, block_mask, window=None, prefix: int = 0,
+            doc=None) -> np.ndarray:
+    """Boolean [len(rows), N]: whether key j is visible to query i.
+
+    Key j is visible to query i iff all of these hold:
+      * right bound: (not causal or j <= i) and, for a sliding window
+        (left, right) with right >= 0, j <= i + right -- unless j < prefix:
+        the first ``prefix`` keys are visible to every query whatever the
+        causal flag and the right bound say (a prefix language model: the
+        prefix attends to itself in both directions);
+      * left bound: for a window with left >= 0, j >= i - left;
+      * documents: ``doc`` (int array [N] of per-token document ids, or None)
+        has doc[j] == doc[i];
+      * block mask: mask[i // 128, j // 128] is non-zero (no mask: all on).
+    A negative window bound means unbounded. The prefix and document rules are
+    mask modifiers in the sense of the lesson's Researcher section ("Beyond
+    hand-written kernels"): one tiled kernel, many masks."""
     rows = np.asarray(rows)
     cols = np.arange(N)
-    ok = np.ones((rows.size, N), dtype=bool)
+    right = np.ones((rows.size, N), dtype=bool)
+    left = np.ones((rows.size, N), dtype=bool)
     if causal:
-        ok &= cols[None, :] <= rows[:, None]
+        right &= cols[None, :] <= rows[:, None]
     if window is not None:
-        left, right = window
-        if left >= 0:
-            ok &= cols[None, :] >= rows[:, None] - left
-        if right >= 0:
-            ok &= cols[None, :] <= rows[:, None] + right
+        wl, wr = window
+        if wl >= 0:
+            left &= cols[None, :] >= rows[:, None] - wl
+        if wr >= 0:
+            right &= cols[None, :] <= rows[:, None] + wr
+    if prefix > 0:
+        right |= cols[None, :] < prefix
+    ok = left & right
+    if doc is not None:
+        doc = np.asarray(doc)
+        ok &= doc[rows][:, None] == doc[None, :N]
     if block_mask is not None:
         ok &= block_mask[(rows // BLOCK)[:, None], (cols // BLOCK)[None, :]].astype(bool)
     return ok
+
+
+def scores(Qr, Kh, scale, softcap: float = 0.0):
+    """Scores of query rows Qr against keys Kh and the scaled products they
+    come from: X = scale * Qr Kh^T, and S = X, or S = softcap * tanh(X / softcap)
+    when softcap > 0 (soft-capping, a score modifier in the FlexAttention
+    sense of the lesson's Researcher section, "Beyond hand-written kernels").
+    Returns (S, X)."""
+    X = scale * (Qr @ Kh.T)
+    if softcap > 0:
+        return softcap * np.tanh(X / softcap), X
+    return X, X
+
+
+def score_grad(dS, X, softcap: float = 0.0):
+    """Chain rule through the score modifier: the gradient with respect to
+    X = scale * Q K^T of a gradient dS with respect to S(X). Soft-capping has
+    dS/dX = 1 - tanh(X / softcap)^2."""
+    if softcap > 0:
+        t = np.tanh(X / softcap)
+        return dS * (1.0 - t * t)
+    return dS
 
 
 def softmax_rows(S: np.ndarray):
@@ -84,8 +126,11 @@ def _kv_head(h: int, Hq: int, Hkv: int) -> int:
     return h // (Hq // Hkv)
 
 
-def forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows, window=None):
-    """O and LSE of query rows ``rows`` of head (b, h), in fp64."""
+def forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows, window=None, prefix=0,
+                 doc=None, softcap=0.0):
+    """O and LSE of query rows ``rows`` of head (b, h), in fp64. The mask and
+    score modifiers (window, prefix, doc, softcap) are those of ``allowed`` and
+    ``scores``; LSE is the logsumexp of the (modified) scores."""
     Hq, Hkv, N = Q.shape[1], K.shape[1], K.shape[2]
     hk = _kv_head(h, Hq, Hkv)
     Kh = K[b, hk].astype(np.float64)
@@ -95,15 +140,16 @@ def forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows, window=None):
     L = np.empty(rows.size)
     for c in range(0, rows.size, ROW_CHUNK):
         r = rows[c:c + ROW_CHUNK]
-        S = scale * (Q[b, h, r].astype(np.float64) @ Kh.T)
-        S[~allowed(r, N, causal, block_mask, window)] = -np.inf
+        S, _ = scores(Q[b, h, r].astype(np.float64), Kh, scale, softcap)
+        S[~allowed(r, N, causal, block_mask, window, prefix, doc)] = -np.inf
         P, lse = softmax_rows(S)
         O[c:c + r.size] = P @ Vh
         L[c:c + r.size] = lse
     return O, L
 
 
-def forward(Q, K, V, scale, causal=False, block_mask=None, window=None):
+def forward(Q, K, V, scale, causal=False, block_mask=None, window=None, prefix=0, doc=None,
+            softcap=0.0):
     """O [B,Hq,N,d] and LSE [B,Hq,N] in fp64 for all heads."""
     B, Hq, N, d = Q.shape
     O = np.empty((B, Hq, N, d))
@@ -112,12 +158,12 @@ def forward(Q, K, V, scale, causal=False, block_mask=None, window=None):
     for b in range(B):
         for h in range(Hq):
             O[b, h], L[b, h] = forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows,
-                                            window)
+                                            window, prefix, doc, softcap)
     return O, L
 
 
 def _head_grads(Qh, Kh, Vh, dOh, Oh, scale, causal, block_mask, rows, want_dq=True,
-                window=None):
+                window=None, prefix=0, doc=None, softcap=0.0):
     """Gradient pieces of one query head restricted to query rows ``rows``.
 
     Returns (dQ_rows or None, dK contribution [N,d], dV contribution [N,d]).
@@ -128,12 +174,12 @@ def _head_grads(Qh, Kh, Vh, dOh, Oh, scale, causal, block_mask, rows, want_dq=Tr
     dQ = np.zeros((rows.size, Qh.shape[1])) if want_dq else None
     for c in range(0, rows.size, ROW_CHUNK):
         r = rows[c:c + ROW_CHUNK]
-        S = scale * (Qh[r] @ Kh.T)
-        S[~allowed(r, N, causal, block_mask, window)] = -np.inf
+        S, X = scores(Qh[r], Kh, scale, softcap)
+        S[~allowed(r, N, causal, block_mask, window, prefix, doc)] = -np.inf
         P, _ = softmax_rows(S)
         dP = dOh[r] @ Vh.T
         D = np.sum(dOh[r] * Oh[r], axis=1)
-        dS = P * (dP - D[:, None])
+        dS = score_grad(P * (dP - D[:, None]), X, softcap)
         dV += P.T @ dOh[r]
         dK += scale * (dS.T @ Qh[r])
         if want_dq:
@@ -141,7 +187,8 @@ def _head_grads(Qh, Kh, Vh, dOh, Oh, scale, causal, block_mask, rows, want_dq=Tr
     return dQ, dK, dV
 
 
-def backward(Q, K, V, dO, scale, causal=False, block_mask=None, O=None, window=None):
+def backward(Q, K, V, dO, scale, causal=False, block_mask=None, O=None, window=None, prefix=0,
+             doc=None, softcap=0.0):
     """dQ [B,Hq,N,d], dK and dV [B,Hkv,N,d] in fp64.
 
     O is the oracle's own forward output (recomputed here when not given).
@@ -149,7 +196,7 @@ def backward(Q, K, V, dO, scale, causal=False, block_mask=None, O=None, window=N
     B, Hq, N, d = Q.shape
     Hkv = K.shape[1]
     if O is None:
-        O, _ = forward(Q, K, V, scale, causal, block_mask, window)
+        O, _ = forward(Q, K, V, scale, causal, block_mask, window, prefix, doc, softcap)
     dQ = np.zeros((B, Hq, N, d))
     dK = np.zeros((B, Hkv, N, d))
     dV = np.zeros((B, Hkv, N, d))
@@ -160,28 +207,32 @@ def backward(Q, K, V, dO, scale, causal=False, block_mask=None, O=None, window=N
             dq, dk, dv = _head_grads(Q[b, h].astype(np.float64), K[b, hk].astype(np.float64),
                                      V[b, hk].astype(np.float64), dO[b, h].astype(np.float64),
                                      O[b, h], scale, causal, block_mask, rows,
-                                     window=window)
+                                     window=window, prefix=prefix, doc=doc, softcap=softcap)
             dQ[b, h] = dq
             dK[b, hk] += dk
             dV[b, hk] += dv
     return dQ, dK, dV
 
 
-def dq_rows(Q, K, V, dO, scale, causal, block_mask, b, h, rows):
+def dq_rows(Q, K, V, dO, scale, causal, block_mask, b, h, rows, window=None, prefix=0,
+            doc=None, softcap=0.0):
     """dQ of query rows ``rows`` of head (b, h) (needs only those rows)."""
     Hq, Hkv = Q.shape[1], K.shape[1]
     hk = _kv_head(h, Hq, Hkv)
     rows = np.asarray(rows)
-    O, _ = forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows)
+    O, _ = forward_rows(Q, K, V, scale, causal, block_mask, b, h, rows, window, prefix, doc,
+                        softcap)
     Oh = np.zeros((Q.shape[2], Q.shape[3]))
     Oh[rows] = O
     dq, _, _ = _head_grads(Q[b, h].astype(np.float64), K[b, hk].astype(np.float64),
                            V[b, hk].astype(np.float64), dO[b, h].astype(np.float64),
-                           Oh, scale, causal, block_mask, rows)
+                           Oh, scale, causal, block_mask, rows, window=window, prefix=prefix,
+                           doc=doc, softcap=softcap)
     return dq
 
 
-def dkdv_rows(Q, K, V, dO, scale, causal, block_mask, b, hk, key_rows):
+def dkdv_rows(Q, K, V, dO, scale, causal, block_mask, b, hk, key_rows, window=None, prefix=0,
+              doc=None, softcap=0.0):
     """dK and dV of key rows ``key_rows`` of KV head (b, hk).
 
     Every query row that can see one of those keys contributes; for each one
@@ -192,8 +243,9 @@ def dkdv_rows(Q, K, V, dO, scale, causal, block_mask, b, hk, key_rows):
     key_rows = np.asarray(key_rows)
     dK = np.zeros((key_rows.size, K.shape[3]))
     dV = np.zeros((key_rows.size, K.shape[3]))
-    vis = allowed(np.arange(N), N, causal, block_mask)[:, key_rows].any(axis=1)
-    qrows = np.flatnonzero(vis)
+    qrows = np.flatnonzero(np.concatenate([
+        allowed(np.arange(c, min(N, c + ROW_CHUNK)), N, causal, block_mask, window, prefix,
+                doc)[:, key_rows].any(axis=1) for c in range(0, N, ROW_CHUNK)]))
     Kh = K[b, hk].astype(np.float64)
     Vh = V[b, hk].astype(np.float64)
     for h in range(hk * g, (hk + 1) * g):
@@ -201,14 +253,14 @@ def dkdv_rows(Q, K, V, dO, scale, causal, block_mask, b, hk, key_rows):
         dOh = dO[b, h].astype(np.float64)
         for c in range(0, qrows.size, ROW_CHUNK):
             r = qrows[c:c + ROW_CHUNK]
-            S = scale * (Qh[r] @ Kh.T)
-            S[~allowed(r, N, causal, block_mask)] = -np.inf
+            S, X = scores(Qh[r], Kh, scale, softcap)
+            S[~allowed(r, N, causal, block_mask, window, prefix, doc)] = -np.inf
             P, _ = softmax_rows(S)
             O = P @ Vh
             D = np.sum(dOh[r] * O, axis=1)
             Pk = P[:, key_rows]
             dPk = dOh[r] @ Vh[key_rows].T
-            dSk = Pk * (dPk - D[:, None])
+            dSk = score_grad(Pk * (dPk - D[:, None]), X[:, key_rows], softcap)
             dV += Pk.T @ dOh[r]
             dK += scale * (dSk.T @ Qh[r])
     return dK, dV

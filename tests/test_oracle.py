@@ -372,3 +372,144 @@ def test_block_mask_recipe():
     nb = 512
     assert m.shape == (nb, nb) and np.all(np.diag(m) == 1)
     assert int(m.sum()) == nb + int(round(0.25 * (nb * nb - nb)))
+
+
+# ---------------------------------------------------------------- mask and score modifiers
+
+def _visible_brute(i, j, causal, window, prefix, doc):
+    """Whether key j is visible to query i, from the modifier rules one by one."""
+    right_ok = (not causal or j <= i)
+    left_ok = True
+    if window is not None:
+        if window[1] >= 0 and j > i + window[1]:
+            right_ok = False
+        if window[0] >= 0 and j < i - window[0]:
+            left_ok = False
+    if j < prefix:
+        right_ok = True
+    return right_ok and left_ok and (doc is None or doc[i] == doc[j])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("window", [None, (5, -1), (3, 2), (-1, 4)])
+@pytest.mark.parametrize("prefix", [0, 1, 7])
+@pytest.mark.parametrize("with_doc", [False, True])
+def test_modifier_visibility_brute_force(causal, window, prefix, with_doc):
+    N = 23
+    doc = np.repeat([0, 1, 2, 3], [6, 1, 9, 7]) if with_doc else None
+    got = orc.allowed(np.arange(N), N, causal, None, window, prefix, doc)
+    for i in range(N):
+        for j in range(N):
+            assert got[i, j] == _visible_brute(i, j, causal, window, prefix, doc), (i, j)
+
+
+def _doc_case(seed, N=150, Hq=2, Hkv=1, d=16):
+    rng = np.random.default_rng(seed)
+    lengths = [37, 1, 64, 48]
+    doc = np.repeat(np.arange(len(lengths)), lengths)
+    assert doc.size == N
+    Q = rng.standard_normal((1, Hq, N, d))
+    K = rng.standard_normal((1, Hkv, N, d))
+    V = rng.standard_normal((1, Hkv, N, d))
+    dO = rng.standard_normal((1, Hq, N, d))
+    return Q, K, V, dO, doc, lengths
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_document_mask_is_attention_per_document(causal):
+    """A document-id mask over packed documents gives, for every document,
+    exactly the attention of that document on its own (forward and
+    gradients)."""
+    Q, K, V, dO, doc, lengths = _doc_case(5)
+    O, L = orc.forward(Q, K, V, 0.3, causal, doc=doc)
+    dQ, dK, dV = orc.backward(Q, K, V, dO, 0.3, causal, doc=doc)
+    s0 = 0
+    for n in lengths:
+        sl = slice(s0, s0 + n)
+        o, lse = orc.forward(Q[:, :, sl], K[:, :, sl], V[:, :, sl], 0.3, causal)
+        dq, dk, dv = orc.backward(Q[:, :, sl], K[:, :, sl], V[:, :, sl], dO[:, :, sl], 0.3, causal)
+        assert np.abs(O[:, :, sl] - o).max() < 1e-12
+        assert np.abs(L[:, :, sl] - lse).max() < 1e-12
+        for a, b_ in ((dQ[:, :, sl], dq), (dK[:, :, sl], dk), (dV[:, :, sl], dv)):
+            assert np.abs(a - b_).max() < 1e-12
+        s0 += n
+
+
+def test_prefix_lm_special_cases():
+    """Prefix LM: a prefix of N or more is full (non-causal) attention, a
+    prefix of 0 or 1 is plain causal attention (key 0 is visible to every
+    query already), and rows inside the prefix see exactly the prefix in both
+    directions (bidirectional attention over the first P tokens alone)."""
+    rng = np.random.default_rng(6)
+    N, d, P = 90, 8, 33
+    Q, K, V = (rng.standard_normal((1, 1, N, d)) for _ in range(3))
+    full, _ = orc.forward(Q, K, V, 0.4, False)
+    causal, _ = orc.forward(Q, K, V, 0.4, True)
+    assert np.abs(orc.forward(Q, K, V, 0.4, True, prefix=N)[0] - full).max() < 1e-12
+    assert np.abs(orc.forward(Q, K, V, 0.4, True, prefix=N + 50)[0] - full).max() < 1e-12
+    for p in (0, 1):
+        assert np.abs(orc.forward(Q, K, V, 0.4, True, prefix=p)[0] - causal).max() < 1e-12
+    O, _ = orc.forward(Q, K, V, 0.4, True, prefix=P)
+    head, _ = orc.forward(Q[:, :, :P], K[:, :, :P], V[:, :, :P], 0.4, False)
+    assert np.abs(O[:, :, :P] - head).max() < 1e-12
+    # a row past the prefix sees keys 0..i: the causal result
+    assert np.abs(O[:, :, P:] - causal[:, :, P:]).max() < 1e-12
+
+
+def test_softcap_limits():
+    """Soft-capping with a huge cap is the plain score; with Q = 0 every score
+    is cap * tanh(0) = 0, so O is the mean of V whatever the cap."""
+    rng = np.random.default_rng(7)
+    Q, K, V = (rng.standard_normal((1, 1, 64, 8)) for _ in range(3))
+    plain, Lp = orc.forward(Q, K, V, 0.5, True)
+    big, Lb = orc.forward(Q, K, V, 0.5, True, softcap=1e7)
+    assert np.abs(plain - big).max() < 1e-9 and np.abs(Lp - Lb).max() < 1e-9
+    O0, _ = orc.forward(np.zeros_like(Q), K, V, 0.5, False, softcap=2.0)
+    assert np.abs(O0[0, 0] - V[0, 0].mean(axis=0)).max() < 1e-12
+
+
+def test_softcap_gradients_finite_differences():
+    """Gradients through the soft-cap chain rule against central differences
+    of sum(O * dO), with a cap small enough to bend the scores."""
+    rng = np.random.default_rng(8)
+    N, d, cap = 9, 4, 1.5
+    Q, K, V, dO = (rng.standard_normal((1, 1, N, d)) * 1.5 for _ in range(4))
+    doc = np.array([0, 0, 0, 0, 1, 1, 1, 1, 1])
+    kw = dict(causal=True, softcap=cap, prefix=2, doc=doc)
+    dQ, dK, dV = orc.backward(Q, K, V, dO, 0.7, **kw)
+
+    def f(Q_, K_, V_):
+        return float(np.sum(orc.forward(Q_, K_, V_, 0.7, **kw)[0] * dO))
+
+    eps = 1e-6
+    for X, G, which in ((Q, dQ, 0), (K, dK, 1), (V, dV, 2)):
+        num = np.zeros_like(X)
+        for idx in np.ndindex(X.shape):
+            Xp, Xm = X.copy(), X.copy()
+            Xp[idx] += eps
+            Xm[idx] -= eps
+            args_p, args_m = [Q, K, V], [Q, K, V]
+            args_p[which], args_m[which] = Xp, Xm
+            num[idx] = (f(*args_p) - f(*args_m)) / (2 * eps)
+        assert np.abs(num - G).max() < 1e-6 * max(1.0, np.abs(G).max())
+
+
+def test_softcap_gradients_match_torch_autograd():
+    """The oracle's hand-derived backward with soft-capping and a document
+    mask equals torch fp64 autograd of the forward formula."""
+    rng = np.random.default_rng(9)
+    N, d, cap, scale = 40, 8, 2.0, 0.6
+    Q, K, V, dO = (rng.standard_normal((1, 1, N, d)) for _ in range(4))
+    doc = np.repeat([0, 1, 2], [10, 18, 12])
+    dQ, dK, dV = orc.backward(Q, K, V, dO, scale, True, softcap=cap, doc=doc)
+    q, k, v = (torch.tensor(a[0, 0], dtype=torch.float64, requires_grad=True) for a in (Q, K, V))
+    x = scale * (q @ k.T)
+    s = cap * torch.tanh(x / cap)
+    i = torch.arange(N)
+    dt = torch.tensor(doc)
+    vis = (i[None, :] <= i[:, None]) & (dt[:, None] == dt[None, :])
+    s = s.masked_fill(~vis, float("-inf"))
+    o = torch.softmax(s, dim=1) @ v
+    (o * torch.tensor(dO[0, 0])).sum().backward()
+    for got, ref in ((dQ, q.grad), (dK, k.grad), (dV, v.grad)):
+        assert np.abs(got[0, 0] - ref.numpy()).max() < 1e-12
