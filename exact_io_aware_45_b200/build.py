@@ -48,16 +48,25 @@ def _stale(target: str, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(verbose_ptxas: bool = False, force: bool = False) -> str:
-    os.makedirs(OUT_DIR, exist_ok=True)
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def build(verbose_ptxas: bool = False, force: bool = False, defines=(), out_dir: str = None) -> str:
+    """Compiles and links libfa.so. ``defines`` are extra ``NAME=VALUE``
+    build-time tuning macros (e.g. FA_FWD_SLOTS_D128=4); a build with defines
+    goes to its own object and output directories (``out_dir``, default
+    ``_build/<defines>/``) so the default library is untouched."""
+    lib_path, build_dir = LIB, BUILD_DIR
+    if defines:
+        tag = "_".join(d.replace("=", "-") for d in defines)
+        build_dir = os.path.join(BUILD_DIR, tag)
+        lib_path = os.path.join(out_dir or build_dir, "libfa.so")
+    os.makedirs(os.path.dirname(lib_path), exist_ok=True)
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdrs = _headers()
     cc = nvcc()
-    extra = ["-Xptxas", "-v"] if verbose_ptxas else []
+    extra = (["-Xptxas", "-v"] if verbose_ptxas else []) + ["-D" + d for d in defines]
 
     def compile_one(src):
-        obj = os.path.join(BUILD_DIR, os.path.basename(src) + ".o")
+        obj = os.path.join(build_dir, os.path.basename(src) + ".o")
         if force or verbose_ptxas or _stale(obj, [src] + hdrs):
             cmd = [cc] + ARCH + FLAGS + extra + ["-c", src, "-o", obj]
             r = subprocess.run(cmd, capture_output=True, text=True)
@@ -69,18 +78,21 @@ def build(verbose_ptxas: bool = False, force: bool = False) -> str:
 
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
         objs = list(ex.map(compile_one, srcs))
-    if force or _stale(LIB, objs):
-        cmd = [cc] + ARCH + ["-shared", "-o", LIB] + objs + ["-lcudart_static", "-ldl",
-                                                             "-lpthread", "-lrt"]
+    if force or _stale(lib_path, objs):
+        cmd = [cc] + ARCH + ["-shared", "-o", lib_path] + objs + ["-lcudart_static", "-ldl",
+                                                                  "-lpthread", "-lrt"]
         r = subprocess.run(cmd, capture_output=True, text=True)
         if r.returncode != 0:
             raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    return LIB
+    return lib_path
 
 
 if __name__ == "__main__":
     ap = argparse.ArgumentParser()
     ap.add_argument("--verbose-ptxas", action="store_true")
     ap.add_argument("--force", action="store_true")
+    ap.add_argument("-D", dest="defines", action="append", default=[],
+                    help="build-time tuning macro NAME=VALUE (separate output directory)")
+    ap.add_argument("--out-dir", default=None)
     a = ap.parse_args()
-    print(build(a.verbose_ptxas, a.force))
+    print(build(a.verbose_ptxas, a.force, tuple(a.defines), a.out_dir))

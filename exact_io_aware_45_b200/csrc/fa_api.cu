@@ -7,6 +7,8 @@
 #include <stdint.h>
 #include <stdio.h>
 
+#include <atomic>
+
 #include "fa.h"
 #include "internal.h"
 
@@ -14,6 +16,16 @@ namespace fa {
 
 static thread_local int t_launches = 0;
 void count_launch(int n) { t_launches += n; }
+
+// Wait-limit test hook (fa_debug_set_stall): kernel families with an injected
+// wait and its limit in SM cycles. Process-wide; read at each launch.
+static std::atomic<int> g_stall_families{0};
+static std::atomic<long long> g_stall_cycles{0};
+long long debug_stall_cycles(int family) {
+  return (g_stall_families.load(std::memory_order_relaxed) & family)
+             ? g_stall_cycles.load(std::memory_order_relaxed)
+             : 0;
+}
 
 namespace {
 
@@ -60,6 +72,45 @@ void fill_common(Problem& p, int B, int Hq, int Hkv, int N, int d, float scale, 
 
 fa_status from_cuda(cudaError_t e) { return e == cudaSuccess ? FA_OK : FA_ERR_CUDA; }
 
+// Mask / score modifiers of a call (fa_mods), validated. `any` is false for a
+// call without modifiers (the plain entry points).
+struct Mods {
+  bool any = false;
+  int wl = -1, wr = -1, prefix = 0;
+  const int* doc = nullptr;
+  float softcap = 0.f;
+};
+
+fa_status read_mods(const fa_mods* m, Mods& out) {
+  out = Mods();
+  if (!m) return FA_OK;
+  if (m->window_left < -1 || m->window_right < -1 || m->prefix < 0) return FA_ERR_INVALID_ARG;
+  if (m->doc_ids && (reinterpret_cast<uintptr_t>(m->doc_ids) & 3u)) return FA_ERR_INVALID_ARG;
+  if (!isfinite(m->softcap) || m->softcap < 0.f) return FA_ERR_INVALID_ARG;
+  out.wl = m->window_left;
+  out.wr = m->window_right;
+  out.prefix = m->prefix;
+  out.doc = m->doc_ids;
+  out.softcap = m->softcap;
+  out.any = out.wl >= 0 || out.wr >= 0 || out.prefix > 0 || out.doc != nullptr ||
+            out.softcap > 0.f;
+  return FA_OK;
+}
+
+// Puts the modifiers into the problem. They run on the tensor-core kernels
+// only: returns false when the caller forced the CUDA-core ones.
+bool apply_mods(const Mods& m, int causal, int& path, Problem& p) {
+  if (!m.any) return true;
+  if (path == FA_PATH_SIMT) return false;
+  path = FA_PATH_TC;
+  p.wl = m.wl;
+  p.wr = causal ? 0 : m.wr;
+  p.prefix = m.prefix;
+  p.doc = m.doc;
+  p.softcap = m.softcap;
+  return true;
+}
+
 }  // namespace
 }  // namespace fa
 
@@ -81,6 +132,16 @@ const char* fa_status_string(int s) {
 int fa_version(void) { return 10000; }
 
 int fa_last_launch_count(void) { return t_launches; }
+
+fa_status fa_debug_set_stall(int kernels, long long wait_cycles) {
+  if (kernels < 0 || kernels > (FA_STALL_FWD | FA_STALL_BWD | FA_STALL_DQ))
+    return FA_ERR_INVALID_ARG;
+  if (kernels != 0 && (wait_cycles < 1000 || wait_cycles > 2000000000ll))
+    return FA_ERR_INVALID_ARG;
+  g_stall_cycles.store(kernels ? wait_cycles : 0);
+  g_stall_families.store(kernels);
+  return FA_OK;
+}
 
 fa_status fa_exp2_fma(const float* x, float* y, long long n, void* stream) {
   t_launches = 0;
@@ -107,8 +168,10 @@ namespace {
 fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                     int Hq, int Hkv, int N, int d, float scale, int causal,
                     const uint8_t* block_mask, int dtype, void* workspace, void* stream,
-                    int path, int wl = -1, int wr = -2) {
+                    int path, const fa_mods* mods = nullptr) {
   t_launches = 0;
+  Mods md;
+  if (fa_status ms = read_mods(mods, md)) return ms;
   fa_status s = check_dims(B, Hq, Hkv, N, d, scale, causal, dtype);
   if (s != FA_OK) return s;
   if (path != FA_PATH_AUTO && path != FA_PATH_SIMT && path != FA_PATH_TC)
@@ -126,14 +189,7 @@ fa_status fwd_impl(const void* Q, const void* K, const void* V, void* O, float* 
   p.Oout = O;
   p.LSEout = LSE;
   p.err = static_cast<unsigned*>(workspace);
-  const bool windowed = wl >= 0 || wr >= -1;
-  if (windowed) {
-    // a window runs on the tensor-core kernels only
-    p.wl = wl;
-    p.wr = causal ? 0 : wr;
-    if (path == FA_PATH_SIMT) return FA_ERR_UNSUPPORTED;
-    path = FA_PATH_TC;
-  }
+  if (!apply_mods(md, causal, path, p)) return FA_ERR_UNSUPPORTED;
   const bool tc_ok = sm100_fwd_supported(p);
   if (path == FA_PATH_TC && !tc_ok) return FA_ERR_UNSUPPORTED;
   const bool use_tc = (path == FA_PATH_TC) || (path == FA_PATH_AUTO && tc_ok);
@@ -158,8 +214,18 @@ fa_status fa_fwd_window(const void* Q, const void* K, const void* V, void* O, fl
                         int window_right, const uint8_t* block_mask, int dtype, void* workspace,
                         void* stream) {
   if (window_left < -1 || window_right < -1) return FA_ERR_INVALID_ARG;
+  // the window call always runs the windowed kernels, also for (-1, -1)
+  fa_mods m = {window_left, window_right, 0, nullptr, 0.f};
   return fwd_impl(Q, K, V, O, LSE, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype, workspace,
-                  stream, FA_PATH_AUTO, window_left, window_right);
+                  stream, FA_PATH_TC, &m);
+}
+
+fa_status fa_fwd_mod(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                     int Hq, int Hkv, int N, int d, float scale, int causal,
+                     const uint8_t* block_mask, const fa_mods* mods, int dtype, void* workspace,
+                     void* stream) {
+  return fwd_impl(Q, K, V, O, LSE, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype, workspace,
+                  stream, FA_PATH_AUTO, mods);
 }
 
 fa_status fa_fwd(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
@@ -181,8 +247,10 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
                    int N, int d, float scale, int causal, const uint8_t* block_mask, int dtype,
                    int grad_dtype, void* workspace, size_t workspace_bytes, void* stream,
                    int path, int stages, const int* cu = nullptr, int total = 0,
-                   int deterministic = 0, int wl = -1, int wr = -2) {
+                   int deterministic = 0, const fa_mods* mods = nullptr) {
   t_launches = 0;
+  Mods md;
+  if (fa_status ms = read_mods(mods, md)) return ms;
   fa_status s = check_dims(B, Hq, Hkv, N, d, scale, causal, dtype);
   if (s != FA_OK) return s;
   if (grad_dtype != FA_F32 && grad_dtype != FA_BF16) return FA_ERR_INVALID_ARG;
@@ -202,13 +270,7 @@ fa_status bwd_impl(const void* Q, const void* K, const void* V, const void* O, c
   fill_common(p, B, Hq, Hkv, N, d, scale, causal, block_mask, dtype, stream);
   p.cu = cu;
   p.total = total;
-  if (wl >= 0 || wr >= -1) {
-    // a window runs on the tensor-core kernels only
-    p.wl = wl;
-    p.wr = causal ? 0 : wr;
-    if (path == FA_PATH_SIMT) return FA_ERR_UNSUPPORTED;
-    path = FA_PATH_TC;
-  }
+  if (!apply_mods(md, causal, path, p)) return FA_ERR_UNSUPPORTED;
   p.Q = Q;
   p.K = K;
   p.V = V;
@@ -305,9 +367,21 @@ fa_status fa_bwd_window(const void* Q, const void* K, const void* V, const void*
                         int window_right, const uint8_t* block_mask, int dtype, int grad_dtype,
                         void* workspace, size_t workspace_bytes, void* stream) {
   if (window_left < -1 || window_right < -1) return FA_ERR_INVALID_ARG;
+  // the window call always runs the windowed kernels, also for (-1, -1)
+  fa_mods m = {window_left, window_right, 0, nullptr, 0.f};
+  return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, Hq, Hkv, N, d, scale, causal, block_mask,
+                  dtype, grad_dtype, workspace, workspace_bytes, stream, FA_PATH_TC, kAll,
+                  nullptr, 0, 0, &m);
+}
+
+fa_status fa_bwd_mod(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                     const float* LSE, void* dQ, void* dK, void* dV, int B, int Hq, int Hkv,
+                     int N, int d, float scale, int causal, const uint8_t* block_mask,
+                     const fa_mods* mods, int dtype, int grad_dtype, void* workspace,
+                     size_t workspace_bytes, void* stream) {
   return bwd_impl(Q, K, V, O, dO, LSE, dQ, dK, dV, B, Hq, Hkv, N, d, scale, causal, block_mask,
                   dtype, grad_dtype, workspace, workspace_bytes, stream, FA_PATH_AUTO, kAll,
-                  nullptr, 0, 0, window_left, window_right);
+                  nullptr, 0, 0, mods);
 }
 
 fa_status fa_bwd_deterministic(const void* Q, const void* K, const void* V, const void* O,

@@ -28,6 +28,14 @@ struct Problem {
   // sliding window: visible keys j of query i satisfy i - wl <= j <= i + wr
   // (-1: unbounded); the launchers apply the causal flag as wr = 0 on top
   int wl = -1, wr = -1;
+  // prefix LM: keys below `prefix` are visible to every query whatever the
+  // right bound says (0: none); doc: [N] non-decreasing per-token document ids
+  // (a query sees only its own document), or null
+  int prefix = 0;
+  const int* doc = nullptr;
+  // soft-capping score modifier: scores x = scale * q.k become
+  // softcap * tanh(x / softcap) (0: off)
+  float softcap = 0.f;
   const uint8_t* mask = nullptr;  // [nb * nb] or null
   int nb = 0;                     // ceil(N / 128)
   int dtype = 0;                  // 0 f32, 1 bf16
@@ -49,6 +57,12 @@ struct Problem {
 
 // Error-word bits set by kernels.
 enum : unsigned { kErrTimeout = 1u, kErrBounds = 2u };
+
+// Kernel families of the wait-limit test hook (fa_debug_set_stall).
+enum : int { kStallFwd = 1, kStallBwd = 2, kStallDq = 4 };
+// Wait limit (SM cycles) of the injected wait of the given family, or 0 when
+// the hook is off for it.
+long long debug_stall_cycles(int family);
 
 // Counts launches made by the current ABI call (thread-local).
 void count_launch(int n = 1);

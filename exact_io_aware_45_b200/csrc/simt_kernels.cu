@@ -15,6 +15,7 @@
 // Idea" item 3). One kernel accumulates dQ over key tiles per query row, a
 // second accumulates dK and dV over query tiles (and over the query heads of a
 // KV group) per key row; neither uses atomics, so the result is deterministic.
+#include <cooperative_groups.h>
 #include <cuda_bf16.h>
 #include <math.h>
 
@@ -24,6 +25,8 @@
 
 namespace fa {
 namespace {
+
+namespace cg = cooperative_groups;
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -61,31 +64,17 @@ __device__ __forceinline__ void load_tile(float (*dst)[D], const T* src, int row
 
 // ------------------------------------------------------------------ forward
 
+// The online-softmax state of one query row over key tiles j0 = k_begin,
+// k_begin + kTile, ... < k_end: running max m (log2 units), sum l and
+// unnormalised output o (this thread's D/4 columns: t * 4 + sub).
 template <int D, typename T>
-__global__ void __launch_bounds__(kThreads) simt_fwd_kernel(Problem p) {
+__device__ __forceinline__ void fwd_key_range(const Problem& p, float (*Ks)[D], float (*Vs)[D],
+                                              const T* Kh, const T* Vh, const float (&q)[D / 4],
+                                              int row, int row0, int sub, int k_begin, int k_end,
+                                              float& m, float& l, float (&o)[D / 4]) {
   constexpr int DT = D / 4;
-  __shared__ float Ks[kTile][D];
-  __shared__ float Vs[kTile][D];
-  const int h = blockIdx.y, b = blockIdx.z;
-  const int hk = h / (p.Hq / p.Hkv);
-  const int row0 = blockIdx.x * kRows;
-  const int row = row0 + threadIdx.x / 4;
-  const int sub = threadIdx.x & 3;
   const int N = p.N;
-  const float c = p.scale * kLog2e;
-  const T* Qh = static_cast<const T*>(p.Q) + ((size_t)b * p.Hq + h) * N * D;
-  const T* Kh = static_cast<const T*>(p.K) + ((size_t)b * p.Hkv + hk) * N * D;
-  const T* Vh = static_cast<const T*>(p.V) + ((size_t)b * p.Hkv + hk) * N * D;
-
-  float q[DT], o[DT];
-#pragma unroll
-  for (int t = 0; t < DT; ++t) {
-    q[t] = (row < N) ? ld<T>(Qh + (size_t)row * D + t * 4 + sub) * c : 0.f;
-    o[t] = 0.f;
-  }
-  float m = -INFINITY, l = 0.f;
-  const int kend = p.causal ? min(N, row0 + kRows) : N;
-  for (int j0 = 0; j0 < kend; j0 += kTile) {
+  for (int j0 = k_begin; j0 < k_end; j0 += kTile) {
     if (p.mask && !p.mask[(size_t)(row0 / 128) * p.nb + j0 / 128]) continue;
     __syncthreads();
     load_tile<D, T>(Ks, Kh, j0, N);
@@ -119,14 +108,120 @@ __global__ void __launch_bounds__(kThreads) simt_fwd_kernel(Problem p) {
     }
     m = m_new;
   }
-  if (row < N) {
-    const size_t base = (((size_t)b * p.Hq + h) * N + row);
-    T* Oh = static_cast<T*>(p.Oout) + base * D;
-    const float inv = (l > 0.f) ? 1.f / l : 0.f;
+}
+
+template <int D, typename T>
+__device__ __forceinline__ void fwd_store_row(const Problem& p, int b, int h, int row, int sub,
+                                              float m, float l, const float (&o)[D / 4]) {
+  if (row >= p.N) return;
+  const size_t base = (((size_t)b * p.Hq + h) * p.N + row);
+  T* Oh = static_cast<T*>(p.Oout) + base * D;
+  const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll
-    for (int t = 0; t < DT; ++t) st<T>(Oh + t * 4 + sub, o[t] * inv);
-    if (sub == 0) p.LSEout[base] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+  for (int t = 0; t < D / 4; ++t) st<T>(Oh + t * 4 + sub, o[t] * inv);
+  if (sub == 0) p.LSEout[base] = (l > 0.f) ? (m + log2f(l)) * kLn2 : -INFINITY;
+}
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kThreads) simt_fwd_kernel(Problem p) {
+  constexpr int DT = D / 4;
+  __shared__ float Ks[kTile][D];
+  __shared__ float Vs[kTile][D];
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / (p.Hq / p.Hkv);
+  const int row0 = blockIdx.x * kRows;
+  const int row = row0 + threadIdx.x / 4;
+  const int sub = threadIdx.x & 3;
+  const int N = p.N;
+  const float c = p.scale * kLog2e;
+  const T* Qh = static_cast<const T*>(p.Q) + ((size_t)b * p.Hq + h) * N * D;
+  const T* Kh = static_cast<const T*>(p.K) + ((size_t)b * p.Hkv + hk) * N * D;
+  const T* Vh = static_cast<const T*>(p.V) + ((size_t)b * p.Hkv + hk) * N * D;
+
+  float q[DT], o[DT];
+#pragma unroll
+  for (int t = 0; t < DT; ++t) {
+    q[t] = (row < N) ? ld<T>(Qh + (size_t)row * D + t * 4 + sub) * c : 0.f;
+    o[t] = 0.f;
   }
+  float m = -INFINITY, l = 0.f;
+  const int kend = p.causal ? min(N, row0 + kRows) : N;
+  fwd_key_range<D, T>(p, Ks, Vs, Kh, Vh, q, row, row0, sub, 0, kend, m, l, o);
+  fwd_store_row<D, T>(p, b, h, row, sub, m, l, o);
+}
+
+// The same forward with the key range of each 32-row query block split over
+// the CTAs of a thread-block cluster (launched with cluster dimension
+// (S, 1, 1), S <= 8): CTA r of the cluster runs the online softmax over its
+// share of the key tiles, and rank 0 merges the S partial states (m_r, l_r,
+// o_r) row by row through distributed shared memory:
+//   m = max_r m_r,  l = sum_r 2^(m_r - m) l_r,  o = sum_r 2^(m_r - m) o_r,
+// the same rescaling the recurrence applies tile by tile. Used when a
+// problem has too few query blocks to fill the GPU (one head of 512 rows is
+// 16 blocks); it needs no global scratch.
+template <int D, typename T>
+__global__ void __launch_bounds__(kThreads) simt_fwd_split_kernel(Problem p) {
+  constexpr int DT = D / 4;
+  static_assert(2 * kTile >= kRows, "partial outputs reuse the K and V tiles");
+  __shared__ float Ks[kTile][D];
+  __shared__ float Vs[kTile][D];
+  __shared__ float part_ml[kRows][2];
+  cg::cluster_group cl = cg::this_cluster();
+  const int S = (int)cl.num_blocks();
+  const int split = (int)cl.block_rank();
+  const int h = blockIdx.y, b = blockIdx.z;
+  const int hk = h / (p.Hq / p.Hkv);
+  const int row0 = (blockIdx.x / S) * kRows;
+  const int r = threadIdx.x / 4;
+  const int row = row0 + r;
+  const int sub = threadIdx.x & 3;
+  const int N = p.N;
+  const float c = p.scale * kLog2e;
+  const T* Qh = static_cast<const T*>(p.Q) + ((size_t)b * p.Hq + h) * N * D;
+  const T* Kh = static_cast<const T*>(p.K) + ((size_t)b * p.Hkv + hk) * N * D;
+  const T* Vh = static_cast<const T*>(p.V) + ((size_t)b * p.Hkv + hk) * N * D;
+
+  float q[DT], o[DT];
+#pragma unroll
+  for (int t = 0; t < DT; ++t) {
+    q[t] = (row < N) ? ld<T>(Qh + (size_t)row * D + t * 4 + sub) * c : 0.f;
+    o[t] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  const int kend = p.causal ? min(N, row0 + kRows) : N;
+  const int ntile = (kend + kTile - 1) / kTile;
+  const int t0 = (int)((long long)split * ntile / S), t1 = (int)((long long)(split + 1) * ntile / S);
+  fwd_key_range<D, T>(p, Ks, Vs, Kh, Vh, q, row, row0, sub, t0 * kTile, min(kend, t1 * kTile), m,
+                      l, o);
+  // partial state into this CTA's shared memory (o over the K/V tiles)
+  __syncthreads();
+  float* po = &Ks[0][0];   // [kRows][D]
+#pragma unroll
+  for (int t = 0; t < DT; ++t) po[r * D + t * 4 + sub] = o[t];
+  if (sub == 0) {
+    part_ml[r][0] = m;
+    part_ml[r][1] = l;
+  }
+  cl.sync();
+  if (split == 0) {
+    float mm = -INFINITY;
+    for (int s = 0; s < S; ++s) mm = fmaxf(mm, cl.map_shared_rank(&part_ml[0][0], s)[2 * r]);
+    float ls = 0.f, os[DT];
+#pragma unroll
+    for (int t = 0; t < DT; ++t) os[t] = 0.f;
+    if (mm != -INFINITY) {
+      for (int s = 0; s < S; ++s) {
+        const float* ml = cl.map_shared_rank(&part_ml[0][0], s);
+        const float* ps = cl.map_shared_rank(po, s);
+        const float w = exp2f(ml[2 * r] - mm);   // 0 for a split that saw nothing
+        ls = fmaf(w, ml[2 * r + 1], ls);
+#pragma unroll
+        for (int t = 0; t < DT; ++t) os[t] = fmaf(w, ps[r * D + t * 4 + sub], os[t]);
+      }
+    }
+    fwd_store_row<D, T>(p, b, h, row, sub, mm, ls, os);
+  }
+  cl.sync();   // the other CTAs' shared memory stays alive until rank 0 has read it
 }
 
 // ------------------------------------------------------------------ backward
@@ -344,8 +439,33 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float* __restrict
 
 template <int D, typename T>
 cudaError_t launch_fwd(const Problem& p) {
-  dim3 grid((p.N + kRows - 1) / kRows, p.Hq, p.B);
-  simt_fwd_kernel<D, T><<<grid, kThreads, 0, p.stream>>>(p);
+  const long long nblk = (p.N + kRows - 1) / kRows;
+  const long long blocks = nblk * p.Hq * p.B;
+  // Too few query blocks to fill the 148 SMs: split each block's key tiles
+  // over a cluster of S CTAs (S a power of two, at most 8 and at most the
+  // block's key tiles), merged through distributed shared memory.
+  int S = 1;
+  const long long ktiles = (p.N + kTile - 1) / kTile;
+  while (S < 8 && blocks * S < 148 && 2 * S <= ktiles) S *= 2;
+  if (S == 1) {
+    dim3 grid((unsigned)nblk, p.Hq, p.B);
+    simt_fwd_kernel<D, T><<<grid, kThreads, 0, p.stream>>>(p);
+  } else {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(nblk * S), p.Hq, p.B);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = p.stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = S;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, simt_fwd_split_kernel<D, T>, p);
+    if (e != cudaSuccess) return e;
+  }
   count_launch();
   return cudaGetLastError();
 }

@@ -50,15 +50,31 @@ using namespace sm100;
 
 constexpr int kBN = 128;            // keys per CTA
 constexpr int kMaxQTiles = 4096;    // query tiles per sequence
-constexpr int kChunk = 8;           // KV heads interleaved in launch order
+// KV heads interleaved in launch order (build-time tuning; default measured
+// on B200)
+#ifndef FA_BWD_CHUNK
+#define FA_BWD_CHUNK 8
+#endif
+constexpr int kChunk = FA_BWD_CHUNK;
+// 1: at d = 128 the two softmax warpgroups take alternate items (build-time
+// choice for A/B measurements; 0: one warpgroup takes every item).
+#ifndef FA_BWD_ITEM_SPLIT
+#define FA_BWD_ITEM_SPLIT 1
+#endif
 constexpr float kLog2e = 1.4426950408889634f;
 
 template <int D>
 struct Cfg {
-  // Softmax / dS warps: 8 (two per TMEM lane quarter, each on half of the
-  // query columns) for d = 64, where that measured 17% faster on B200; 4 for
-  // d = 128, where the split measured 3% slower.
-  static constexpr int kSoftWarps = (D == 64) ? 8 : 4;
+  // Softmax / dS warps, in groups of four (one warp per TMEM lane quarter).
+  // d = 64: two groups, each on half of every item's query columns (measured
+  // 17% faster on B200 than one group). d = 128: two groups taking alternate
+  // items, each on its own S^T / dP^T set in TMEM, dS^T buffer and p_ready
+  // barrier, so the softmax of two items runs at once (one group on every
+  // item left the MMA warp waiting: the per-item softmax / dS step is
+  // latency-bound at one warp per SMSP).
+  static constexpr bool kItemSplit = (D == 128) && FA_BWD_ITEM_SPLIT;
+  static constexpr int kSoftWarps = (D == 64 || kItemSplit) ? 8 : 4;
+  static constexpr int kColHalves = (D == 64) ? 2 : 1;    // groups sharing an item's columns
   static constexpr int kThreads = (8 + kSoftWarps) * 32;
   static constexpr bool kDbl = (D == 128);                // two S/dP sets in TMEM
   static constexpr int MQ = (D == 64) ? 128 : 64;         // query rows per item
@@ -91,11 +107,17 @@ struct alignas(16) Ctl {
   uint64_t kv_full;
   uint64_t qdo_full[3], qdo_empty[3];
   uint64_t sp_full[2], p_ready[2], dq_full, dq_free, acc_done;
+  uint64_t never;              // signalled by nothing (wait-limit test hook)
   uint32_t tmem_base;
   int abort;
+  int skip;                    // the error word was set at launch: the CTA does nothing
   int nq;                      // visible query tiles per query head
-  uint16_t qtiles[kMaxQTiles];
+  uint16_t qtiles[kMaxQTiles];  // visible query tiles, | kFullBit
 };
+
+// Flag on a query-tile entry: every (query, key) pair of the item is
+// visible, so its scores need no masking.
+constexpr uint16_t kFullBit = 0x8000;
 
 struct BwdParams {
   CUtensorMap tq, tdo;         // [B*Hq][N][d] bf16, box {64, MQ}, 128B swizzle
@@ -108,12 +130,14 @@ struct BwdParams {
   const uint8_t* mask;
   unsigned* err;
   int N, Npad, Hq, Hkv, nb, causal, grad_bf16, BHk;
-  int wl, wr;                  // visible keys: row - wl <= key <= row + wr (-1: unbounded)
+  MaskMod mod;                 // keys each query sees (the causal flag is its wr = 0)
   float c;                     // scale * log2(e)
+  float cap1, cap2;            // soft-capping: scores in log2 units = cap1 * tanh(cap2 * q.k)
   float scale;
   const int* cu;               // variable-length batch: sequence offsets [B+1], or null
   int total;                   // packed rows (variable-length batch)
   int no_dq;                   // skip dQ (the deterministic dQ kernel computes it)
+  long long stall;             // > 0: injected wait of this many cycles (test hook)
 };
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -123,7 +147,7 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int D, bool kVarlen>
+template <int D, bool kVarlen, bool kCap>
 __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_constant__ BwdParams p) {
   using C = Cfg<D>;
   constexpr int MQ = C::MQ;
@@ -141,7 +165,11 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   chunked_order(blockIdx.x, p.nb, p.BHk, kChunk, bhk, kb);
   // A launch whose error word is already set (an earlier wait ran out and
   // nobody has read the word yet) does no work: its inputs may be invalid.
-  if (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) return;
+  // One thread reads the word and the whole CTA leaves together, before any
+  // barrier is initialised or TMEM allocated.
+  if (threadIdx.x == 0) ctl.skip = (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) ? 1 : 0;
+  __syncthreads();
+  if (ctl.skip) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = kb * kBN;
   const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
@@ -167,11 +195,12 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
     }
     mbar_init(&ctl.sp_full[0], 1);
     mbar_init(&ctl.sp_full[1], 1);
-    mbar_init(&ctl.p_ready[0], C::kSoftWarps);
-    mbar_init(&ctl.p_ready[1], C::kSoftWarps);
+    mbar_init(&ctl.p_ready[0], C::kItemSplit ? 4 : C::kSoftWarps);
+    mbar_init(&ctl.p_ready[1], C::kItemSplit ? 4 : C::kSoftWarps);
     mbar_init(&ctl.dq_full, 1);
     mbar_init(&ctl.dq_free, 4);
     mbar_init(&ctl.acc_done, 1);
+    mbar_init(&ctl.never, 1);
     ctl.abort = 0;
     fence_mbar_init();
   }
@@ -180,17 +209,22 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
     tmem_relinquish();
   }
   if (warp == 3) {
-    // Query tiles that can see this key tile, in increasing order.
+    // Query tiles that can see this key tile, in increasing order (entries
+    // flagged kFullBit see all of it).
     const int nqt = (N + MQ - 1) / MQ;
-    // first query tile whose last row reaches the window of this key tile
-    const int qt_lo = p.wr >= 0 ? max(0, (n0 - p.wr) / MQ) : 0;
+    // first query tile whose rows can reach this key tile
+    const int qt_lo = mod_first_query(p.mod, n0) / MQ;
     int count = 0;
     for (int t0 = qt_lo; t0 < nqt; t0 += 32) {
       const int qt = t0 + lane;
-      const bool vis = qt < nqt && (!p.mask || p.mask[(size_t)((qt * MQ) / 128) * p.nb + kb]) &&
-                       win_any(qt * MQ, qt * MQ + MQ - 1, n0, n0 + kBN - 1, p.wl, p.wr);
+      int cls = kTileEmpty;
+      if (qt < nqt && (!p.mask || p.mask[(size_t)((qt * MQ) / 128) * p.nb + kb]))
+        cls = mod_classify(p.mod, qt * MQ, qt * MQ + MQ - 1, n0, n0 + kBN - 1, N);
+      const bool vis = cls != kTileEmpty;
       const unsigned bal = __ballot_sync(0xffffffffu, vis);
-      if (vis) ctl.qtiles[count + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(qt);
+      if (vis)
+        ctl.qtiles[count + __popc(bal & ((1u << lane) - 1u))] =
+            static_cast<uint16_t>(qt | (cls == kTileFull ? kFullBit : 0));
       count += __popc(bal);
     }
     if (lane == 0) ctl.nq = count;
@@ -202,13 +236,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   const int nq = ctl.nq;
   const int n_items = nq * grp;
   const Guard g{&ctl.abort, p.err};
-  constexpr int kChunks = MQ / 32 / (C::kSoftWarps / 4);   // 32-column chunks per softmax warp
+  constexpr int kChunks = MQ / 32 / C::kColHalves;   // 32-column chunks per softmax warp
   static_assert(kChunks == 2, "the MMA warp waits on two chunk steps per item");
   // item i -> (query head, first query row)
   auto item_bh = [&](int i) { return b * p.Hq + hk * grp + i / nq; };
   // TMA plane of item i's Q / dO / dQ rows
   auto item_plane = [&](int i) { return kVarlen ? hk * grp + i / nq : item_bh(i); };
-  auto item_q0 = [&](int i) { return static_cast<int>(ctl.qtiles[i % nq]) * MQ; };
+  auto item_q0 = [&](int i) { return static_cast<int>(ctl.qtiles[i % nq] & ~kFullBit) * MQ; };
   // TMEM columns of item i
   auto s_col = [&](int i) { return (i & 1) ? C::kS1 : C::kS0; };
   auto dp_col = [&](int i) { return (i & 1) ? C::kDP1 : C::kDP0; };
@@ -285,7 +319,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       auto issue_dv = [&](int i, int st) {  // P^T bf16 in the S columns
         const uint32_t dos = dostage(i);
 #pragma unroll
-        for (int h = 0; h < C::kSoftWarps / 4; ++h)
+        for (int h = 0; h < C::kColHalves; ++h)
 #pragma unroll
           for (int k2 = 0; k2 < 2; ++k2) {
             const int kk = 2 * (h * kChunks + st) + k2;
@@ -296,7 +330,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       auto issue_dk = [&](int i, int st) {
         const uint32_t qs = qstage(i), dsb = dsbuf(i);
 #pragma unroll
-        for (int h = 0; h < C::kSoftWarps / 4; ++h)
+        for (int h = 0; h < C::kColHalves; ++h)
 #pragma unroll
           for (int k2 = 0; k2 < 2; ++k2) {
             const int kk = 2 * (h * kChunks + st) + k2;
@@ -320,7 +354,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       auto wait_q = [&](int i) {
         return mbar_wait(&ctl.qdo_full[i % C::kStages], (i / C::kStages) & 1, g);
       };
-      bool ok = mbar_wait(&ctl.kv_full, 0, g) && wait_q(0);
+      bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait(&ctl.kv_full, 0, g) &&
+                wait_q(0);
       if (ok) {
         tc_fence_after();
         issue_s(0);
@@ -393,15 +428,21 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
     }
   } else if (warp >= 4 && warp < 4 + C::kSoftWarps) {
     // ------------------------------------------------------------ softmax / dS
-    // With 8 softmax warps, warps 4-7 take the first half of each item's
-    // query columns and warps 8-11 the second half; with 4, warps 4-7 take all.
+    // d = 64: warps 4-7 take the first half of each item's query columns and
+    // warps 8-11 the second half. d = 128: warps 4-7 take the even items and
+    // warps 8-11 the odd ones (with FA_BWD_ITEM_SPLIT=0, warps 4-7 take all).
     const int wq = warp & 3;
     const int half = (warp - 4) >> 2;
+    const int i_first = C::kItemSplit ? half : 0, i_step = C::kItemSplit ? 2 : 1;
+    const int col_half = C::kItemSplit ? 0 : half;
     const int r = wq * 32 + lane;                 // key row inside the tile
     const int kv = n0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const float c = p.c;
-    for (int i = 0; i < n_items; ++i) {
+    // queries that see this thread's key: [qlo, qhi] (empty past N)
+    int qlo, qhi;
+    mod_key_queries(p.mod, kv, N, qlo, qhi);
+    for (int i = i_first; i < n_items; i += i_step) {
       const int s = i % C::kStages;
       const bool spok = C::kDbl ? mbar_wait(&ctl.sp_full[i & 1], (i >> 1) & 1, g)
                                 : mbar_wait(&ctl.sp_full[0], i & 1, g);
@@ -409,17 +450,13 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       if (!mbar_wait(&ctl.qdo_full[s], (i / C::kStages) & 1, g)) break;
       tc_fence_after();
       const int q0 = item_q0(i);
-      const bool need_mask =
-          kv >= N || win_cuts(q0, q0 + MQ - 1, n0, n0 + kBN - 1, p.wl, p.wr);
-      // queries that see this thread's key: [qlo, qhi] (empty past N)
-      const int qlo = (p.wr >= 0) ? kv - p.wr : 0;
-      const int qhi = (kv >= N) ? -1 : ((p.wl >= 0) ? kv + p.wl : 0x7fffffff);
+      const bool need_mask = !(ctl.qtiles[i % nq] & kFullBit);
       const float* lse_s = vec + (s * 2 + 0) * MQ;
       const float* d_s = vec + (s * 2 + 1) * MQ;
       uint8_t* dsrow = base + C::kOffDS + (i & 1) * C::kDSBytes + r * 128;
 #pragma unroll 1
       for (int ch = 0; ch < kChunks; ++ch) {
-        const int cc = half * kChunks + ch;
+        const int cc = col_half * kChunks + ch;
         uint32_t sv[32], dp[32];
         tmem_ld32x2(tm + s_col(i) + lane_off + cc * 32, tm + dp_col(i) + lane_off + cc * 32, sv,
                     dp);
@@ -431,14 +468,26 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
           const float4 dd = *reinterpret_cast<const float4*>(d_s + ((cc * 32 + e) & ~3));
           const float la = (e & 2) ? l2.z : l2.x, lb = (e & 2) ? l2.w : l2.y;
           const float da_ = (e & 2) ? dd.z : dd.x, db_ = (e & 2) ? dd.w : dd.y;
-          float p0 = ex2(fmaf(__uint_as_float(sv[e]), c, -la));
-          float p1 = ex2(fmaf(__uint_as_float(sv[e + 1]), c, -lb));
+          // soft-capping: P from the capped score, and dS picks up the
+          // derivative of the cap, 1 - tanh^2
+          float t0 = 0.f, t1 = 0.f;
+          if constexpr (kCap) {
+            t0 = tanh_ex2(__uint_as_float(sv[e]) * p.cap2);
+            t1 = tanh_ex2(__uint_as_float(sv[e + 1]) * p.cap2);
+          }
+          float p0 = kCap ? ex2(fmaf(t0, p.cap1, -la)) : ex2(fmaf(__uint_as_float(sv[e]), c, -la));
+          float p1 =
+              kCap ? ex2(fmaf(t1, p.cap1, -lb)) : ex2(fmaf(__uint_as_float(sv[e + 1]), c, -lb));
           if (need_mask) {
             if (qa_ < qlo || qa_ > qhi) p0 = 0.f;
             if (qa_ + 1 < qlo || qa_ + 1 > qhi) p1 = 0.f;
           }
-          const float g0 = p0 * (__uint_as_float(dp[e]) - da_);
-          const float g1 = p1 * (__uint_as_float(dp[e + 1]) - db_);
+          float g0 = p0 * (__uint_as_float(dp[e]) - da_);
+          float g1 = p1 * (__uint_as_float(dp[e + 1]) - db_);
+          if constexpr (kCap) {
+            g0 *= fmaf(-t0, t0, 1.f);
+            g1 *= fmaf(-t1, t1, 1.f);
+          }
           pk[e >> 1] = pack_bf16(p0, p1);
           dk[e >> 1] = pack_bf16(g0, g1);
         }
@@ -458,7 +507,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
         // item i+1's S is issued only after both steps of item i, so no warp
         // runs an item ahead); for d = 128 it waits for the whole item (one
         // signal after the last chunk, on p_ready[i & 1]).
-        if (C::kSoftWarps == 8 || ch == kChunks - 1) {
+        if (C::kColHalves == 2 || ch == kChunks - 1) {
           tmem_st_wait();
           fence_async_smem();
           tc_fence_before();
@@ -616,32 +665,33 @@ cudaError_t launch(const Problem& pr) {
   kp.Hkv = pr.Hkv;
   kp.nb = pr.nb;
   kp.causal = pr.causal;
-  // a bound of N or more cuts nothing: unbounded (keeps row +- bound in int range)
-  kp.wl = (pr.wl >= pr.N) ? -1 : pr.wl;
-  kp.wr = pr.causal ? 0 : ((pr.wr >= pr.N) ? -1 : pr.wr);   // causal is the window wr = 0
+  kp.mod = mask_mod_of(pr);
+  kp.cap1 = pr.softcap > 0.f ? pr.softcap * kLog2e : 0.f;
+  kp.cap2 = pr.softcap > 0.f ? pr.scale / pr.softcap : 0.f;
   kp.grad_bf16 = pr.grad_dtype == 1;
   kp.c = pr.scale * kLog2e;
   kp.scale = pr.scale;
   kp.cu = pr.cu;
   kp.total = pr.total;
   kp.no_dq = pr.no_dq;
+  kp.stall = debug_stall_cycles(kStallBwd);
   const size_t smem = sizeof(Ctl) + 1024 + C::kOffEnd;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(bwd_kernel<D, false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(bwd_kernel<D, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)smem);
+  for (const void* f : {(const void*)bwd_kernel<D, false, false>,
+                        (const void*)bwd_kernel<D, true, false>,
+                        (const void*)bwd_kernel<D, false, true>}) {
+    const cudaError_t e = set_max_dynamic_smem(f, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   kp.BHk = (int)BHk;
   dim3 grid((unsigned)(BHk * pr.nb));
+  const bool cap = pr.softcap > 0.f;
+  if (pr.cu && cap) return cudaErrorInvalidValue;   // not offered for packed batches
   if (pr.cu)
-    bwd_kernel<D, true><<<grid, C::kThreads, smem, pr.stream>>>(kp);
+    bwd_kernel<D, true, false><<<grid, C::kThreads, smem, pr.stream>>>(kp);
+  else if (cap)
+    bwd_kernel<D, false, true><<<grid, C::kThreads, smem, pr.stream>>>(kp);
   else
-    bwd_kernel<D, false><<<grid, C::kThreads, smem, pr.stream>>>(kp);
+    bwd_kernel<D, false, false><<<grid, C::kThreads, smem, pr.stream>>>(kp);
   count_launch();
   return cudaGetLastError();
 }

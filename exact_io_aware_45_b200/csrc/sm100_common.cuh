@@ -74,6 +74,16 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
+// tanh(u) = 1 - 2 / (1 + e^(2u)) from the MUFU base-2 exponential and a fast
+// reciprocal; absolute error about 1e-7 (u is clamped to [-20, 20], where
+// tanh is +-1 to float precision, so the exponential stays finite). Used by
+// the soft-capping score modifier.
+__device__ __forceinline__ float tanh_ex2(float u) {
+  u = fminf(fmaxf(u, -20.f), 20.f);
+  const float e = ex2(u * 2.8853900817779268f);   // 2 log2(e)
+  return 1.f - __fdividef(2.f, 1.f + e);
+}
+
 // Named barrier among `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -127,15 +137,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete. Returns false if the
-// CTA has aborted or the wait ran out (which then aborts the CTA).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Guard& g) {
+// CTA has aborted or the wait ran out (which then aborts the CTA). `limit` is
+// the wait limit in SM clock cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const Guard& g,
+                                          long long limit = kWaitLimitCycles) {
   if (*g.abort) return false;
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*g.abort) return false;
-    if (clock64() - t0 > kWaitLimitCycles) {
+    if (clock64() - t0 > limit) {
       *g.abort = 1;
       atomicOr(g.err, kErrTimeout);
       __threadfence();
@@ -144,19 +156,125 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
-// Visibility of key j to query i under a window (FlexAttention-style mask
-// modifier): i - wl <= j <= i + wr, a negative bound meaning unbounded. The
-// causal flag is the window wr = 0, wl unbounded.
-__device__ __forceinline__ bool win_ok(int i, int j, int wl, int wr) {
-  return (wr < 0 || j <= i + wr) && (wl < 0 || j >= i - wl);
+// Test hook of the bounded-wait contract: when stall_cycles > 0 the caller
+// waits on `never`, a barrier initialised with one expected arrival that
+// nothing ever signals, with that short limit. The wait runs out and takes
+// the normal abort path (error word set, every other wait of the CTA returns
+// at once, in-flight copies and MMAs are drained, TMEM is freed). Returns
+// false after such a stall; true (without waiting) when stall_cycles <= 0.
+__device__ __forceinline__ bool injected_stall(uint64_t* never, long long stall_cycles,
+                                               const Guard& g) {
+  if (stall_cycles <= 0) return true;
+  return mbar_wait(never, 0, g, stall_cycles);
 }
-// Some pair of query rows [r0, r1] and keys [c0, c1] is visible.
-__device__ __forceinline__ bool win_any(int r0, int r1, int c0, int c1, int wl, int wr) {
-  return (wr < 0 || c0 <= r1 + wr) && (wl < 0 || c1 >= r0 - wl);
+
+// ---------------------------------------------------------------- mask modifiers
+
+// Which keys a query sees, before the 128 x 128 block mask (a mask modifier
+// in the FlexAttention sense: one tiled kernel, many masks). Key j is visible
+// to query i iff lo(i) <= j <= hi(i), where
+//   hi(i) = min(wr >= 0 ? max(i + wr, prefix - 1) : N - 1, last row of i's document)
+//   lo(i) = max(wl >= 0 ? i - wl : 0, first row of i's document)
+// The causal flag is the window wr = 0; prefix > 0 makes the first `prefix`
+// keys visible to every query whatever the right bound says (prefix LM);
+// doc lists one document id per token, non-decreasing, and a query sees only
+// its own document. lo and hi are non-decreasing in i, so the queries that see
+// key j form an interval too, and the visibility of a tile follows from its
+// corner rows and columns.
+struct MaskMod {
+  int wl, wr;          // window bounds, -1 unbounded (the causal flag sets wr = 0)
+  int prefix;          // keys below this are visible to every query (0: none)
+  const int* doc;      // [N] non-decreasing document ids, or null
+};
+
+// First and last row of the run of equal ids that contains row i (binary
+// searches over [0, i] and [i, N - 1]). Ids that are not sorted give wrong
+// runs but no access outside doc[0 .. N-1].
+__device__ __forceinline__ int doc_first(const int* doc, int i) {
+  const int t = doc[i];
+  int a = 0, b = i;
+  while (a < b) {
+    const int mid = (a + b) >> 1;
+    if (doc[mid] < t) a = mid + 1; else b = mid;
+  }
+  return a;
 }
-// Some pair of query rows [r0, r1] and keys [c0, c1] is hidden by the window.
-__device__ __forceinline__ bool win_cuts(int r0, int r1, int c0, int c1, int wl, int wr) {
-  return (wr >= 0 && c1 > r0 + wr) || (wl >= 0 && c0 < r1 - wl);
+__device__ __forceinline__ int doc_last(const int* doc, int i, int N) {
+  const int t = doc[i];
+  int a = i, b = N - 1;
+  while (a < b) {
+    const int mid = (a + b + 1) >> 1;
+    if (doc[mid] > t) b = mid - 1; else a = mid;
+  }
+  return a;
+}
+
+// Keys [lo, hi] that query row i sees (empty when lo > hi). Rows at or past N
+// get the interval of row N - 1 (their results are never stored).
+__device__ __forceinline__ void mod_row_keys(const MaskMod& m, int i, int N, int& lo, int& hi) {
+  hi = N - 1;
+  lo = 0;
+  if (m.wr >= 0) hi = min(hi, max(i + m.wr, m.prefix - 1));
+  if (m.wl >= 0) lo = max(0, i - m.wl);
+  if (m.doc) {
+    const int r = min(i, N - 1);
+    lo = max(lo, doc_first(m.doc, r));
+    hi = min(hi, doc_last(m.doc, r, N));
+  }
+}
+
+// Queries [qlo, qhi] that see key j (empty when qlo > qhi; keys at or past N
+// see nothing).
+__device__ __forceinline__ void mod_key_queries(const MaskMod& m, int j, int N, int& qlo,
+                                                int& qhi) {
+  qlo = 0;
+  qhi = N - 1;
+  if (j >= N) {
+    qhi = -1;
+    return;
+  }
+  if (m.wr >= 0 && j >= m.prefix) qlo = max(0, j - m.wr);
+  if (m.wl >= 0) qhi = min(qhi, j + m.wl);
+  if (m.doc) {
+    qlo = max(qlo, doc_first(m.doc, j));
+    qhi = min(qhi, doc_last(m.doc, j, N));
+  }
+}
+
+enum : int { kTileEmpty = 0, kTilePartial = 1, kTileFull = 2 };
+
+// Visibility of the tile of query rows [r0, r1] and keys [c0, c1] (r0, c0 <
+// N) under the modifier, before the block mask: kTileEmpty if no pair is
+// visible, kTileFull if every pair is (and the tile lies inside the
+// sequence), kTilePartial otherwise. Exact for the window and the prefix;
+// with documents a tile may be called partial although it is empty (its
+// elements are then all masked), never the reverse.
+__device__ __forceinline__ int mod_classify(const MaskMod& m, int r0, int r1, int c0, int c1,
+                                            int N) {
+  const int hi_max = (m.wr >= 0) ? max(r1 + m.wr, m.prefix - 1) : 0x7fffffff;
+  const int lo_min = (m.wl >= 0) ? r0 - m.wl : -0x7fffffff;
+  if (c0 > hi_max || c1 < lo_min) return kTileEmpty;
+  const int hi_min = (m.wr >= 0) ? max(r0 + m.wr, m.prefix - 1) : 0x7fffffff;
+  const int lo_max = (m.wl >= 0) ? r1 - m.wl : -0x7fffffff;
+  bool full = c1 <= hi_min && c0 >= lo_max && r1 < N && c1 < N;
+  if (m.doc) {
+    const int dr0 = m.doc[r0], dr1 = m.doc[min(r1, N - 1)];
+    const int dc0 = m.doc[c0], dc1 = m.doc[min(c1, N - 1)];
+    if (dc1 < dr0 || dc0 > dr1) return kTileEmpty;   // no document in common
+    full = full && dr0 == dr1 && dc0 == dc1 && dr0 == dc0;
+  }
+  return full ? kTileFull : kTilePartial;
+}
+
+// Last key any of the query rows [r0, r1] can see, before documents: the
+// key-tile range of a query block ends there.
+__device__ __forceinline__ int mod_last_key(const MaskMod& m, int r1, int N) {
+  return (m.wr >= 0) ? min(N - 1, max(r1 + m.wr, m.prefix - 1)) : N - 1;
+}
+
+// First query that can see any of the keys [c0, ...], before documents.
+__device__ __forceinline__ int mod_first_query(const MaskMod& m, int c0) {
+  return (m.wr >= 0 && c0 >= m.prefix) ? max(0, c0 - m.wr) : 0;
 }
 
 // Maps a linear CTA index to (head, block) so that the blocks of `chunk`
@@ -453,6 +571,20 @@ bool make_tmap_3d_strided(CUtensorMap* m, const void* base, CUtensorMapDataType 
                           int elem_bytes, uint64_t cols, uint64_t rows, uint64_t planes,
                           uint64_t row_stride, uint64_t plane_stride, uint32_t box_cols,
                           uint32_t box_rows, CUtensorMapSwizzle swz);
+// Sets cudaFuncAttributeMaxDynamicSharedMemorySize of kernel `fn` to `bytes`
+// on the current device, once per (device, kernel, size); thread-safe.
+cudaError_t set_max_dynamic_smem(const void* fn, int bytes);
+// The kernels' mask modifier for a problem: the causal flag becomes the right
+// window bound 0 (it wins over a wider one); a bound of N or more cuts
+// nothing and becomes unbounded (which keeps row +- bound inside int range).
+inline sm100::MaskMod mask_mod_of(const Problem& p) {
+  sm100::MaskMod m;
+  m.wl = (p.wl >= p.N) ? -1 : p.wl;
+  m.wr = p.causal ? 0 : ((p.wr >= p.N) ? -1 : p.wr);
+  m.prefix = (p.prefix > p.N) ? p.N : p.prefix;
+  m.doc = p.doc;
+  return m;
+}
 // The map of a [B][H][N][cols] tensor (dense) or of a packed [total][H][cols]
 // one (variable-length, p.cu set); rows of the box run over N or tokens.
 inline bool make_seq_tmap(CUtensorMap* m, const Problem& p, const void* base,

@@ -55,11 +55,17 @@ struct alignas(16) Ctl {
   uint64_t q_full;
   uint64_t kv_full[4], kv_empty[4];
   uint64_t sp_full, ds_ready, dq_done;
+  uint64_t never;                // signalled by nothing (wait-limit test hook)
   uint32_t tmem_base;
   int abort;
+  int skip;                      // the error word was set at launch: the CTA does nothing
   int ntiles;
-  uint16_t tiles[kMaxTiles];
+  uint16_t tiles[kMaxTiles];     // visible key tiles, | kFullBit
 };
+
+// Flag on a key-tile entry: every (query, key) pair of the tile is visible,
+// so its scores need no masking.
+constexpr uint16_t kFullBit = 0x8000;
 
 struct DqParams {
   CUtensorMap tq, tdo, tk, tv;   // [B*H][N][d] bf16, box {64, 128, 1}, 128B swizzle
@@ -69,9 +75,10 @@ struct DqParams {
   const uint8_t* mask;
   unsigned* err;
   int N, Npad, Hq, Hkv, nb, nqt, causal, BH, grad_bf16;
-  int wl, wr;                    // visible keys: row - wl <= key <= row + wr (-1: unbounded)
+  MaskMod mod;                   // keys each query sees (the causal flag is its wr = 0)
   float c;                       // scale * log2(e)
   float scale;
+  long long stall;               // > 0: injected wait of this many cycles (test hook)
 };
 
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -94,7 +101,12 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
   // tiles (the last ones under the causal flag) start first.
   int bh, rqt;
   chunked_order(blockIdx.x, p.nqt, p.BH, kChunk, bh, rqt);
-  if (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) return;
+  // A launch whose error word is already set does no work; one thread reads
+  // the word and the whole CTA leaves together, before any barrier is
+  // initialised or TMEM allocated.
+  if (threadIdx.x == 0) ctl.skip = (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) ? 1 : 0;
+  __syncthreads();
+  if (ctl.skip) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int qt = p.nqt - 1 - rqt;
   const int q0 = qt * kBM;
@@ -111,6 +123,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     mbar_init(&ctl.sp_full, 1);
     mbar_init(&ctl.ds_ready, 4);
     mbar_init(&ctl.dq_done, 1);
+    mbar_init(&ctl.never, 1);
     ctl.abort = 0;
     fence_mbar_init();
   }
@@ -119,15 +132,20 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     tmem_relinquish();
   }
   if (warp == 3) {
-    // Key tiles this query tile sees, in increasing order.
-    const int kb_end = p.wr >= 0 ? min(p.nb, (q0 + kBM - 1 + p.wr) / kBN + 1) : p.nb;
+    // Key tiles this query tile sees, in increasing order (entries flagged
+    // kFullBit are seen whole).
+    const int kb_end = min(p.nb, mod_last_key(p.mod, q0 + kBM - 1, N) / kBN + 1);
     int count = 0;
     for (int kb0 = 0; kb0 < kb_end; kb0 += 32) {
       const int kb = kb0 + lane;
-      const bool act = kb < kb_end && (!p.mask || p.mask[(size_t)qt * p.nb + kb]) &&
-                       win_any(q0, q0 + kBM - 1, kb * kBN, kb * kBN + kBN - 1, p.wl, p.wr);
+      int cls = kTileEmpty;
+      if (kb < kb_end && (!p.mask || p.mask[(size_t)qt * p.nb + kb]))
+        cls = mod_classify(p.mod, q0, q0 + kBM - 1, kb * kBN, kb * kBN + kBN - 1, N);
+      const bool act = cls != kTileEmpty;
       const unsigned bal = __ballot_sync(0xffffffffu, act);
-      if (act) ctl.tiles[count + __popc(bal & ((1u << lane) - 1u))] = static_cast<uint16_t>(kb);
+      if (act)
+        ctl.tiles[count + __popc(bal & ((1u << lane) - 1u))] =
+            static_cast<uint16_t>(kb | (cls == kTileFull ? kFullBit : 0));
       count += __popc(bal);
     }
     if (lane == 0) ctl.ntiles = count;
@@ -158,7 +176,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         const int s = j % C::kStages;
         if (j >= C::kStages && !mbar_wait(&ctl.kv_empty[s], ((j / C::kStages) - 1) & 1, g))
           break;
-        const int kb = ctl.tiles[j];
+        const int kb = ctl.tiles[j] & ~kFullBit;
         mbar_expect_tx(&ctl.kv_full[s], 2 * C::kTileBytes);
         for (int cb = 0; cb < C::kColBlocks; ++cb) {
           tma_load_3d(tiles_base + C::kOffK + s * C::kTileBytes + cb * C::kBlockBytes, &p.tk,
@@ -190,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
                  kk > 0);
         }
       };
-      bool ok = mbar_wait(&ctl.q_full, 0, g);
+      bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait(&ctl.q_full, 0, g);
       for (int j = 0; ok && j < T; ++j) {
         const int s = j % C::kStages;
         if (!(ok = mbar_wait(&ctl.kv_full[s], (j / C::kStages) & 1, g))) break;
@@ -220,15 +238,16 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     const float c = p.c;
     const size_t vrow = (size_t)bh * p.Npad + row;   // padded: row < Npad always
     const float lse2 = p.lse2[vrow], dd = p.dvec[vrow];
+    // this row's visible keys: [klo, khi] (empty past N)
+    int klo, khi;
+    mod_row_keys(p.mod, row, N, klo, khi);
+    if (row >= N) khi = -1;
     for (int j = 0; j < T; ++j) {
       if (!mbar_wait(&ctl.sp_full, j & 1, g)) break;
       tc_fence_after();
-      const int col0 = ctl.tiles[j] * kBN;
-      const bool need_mask = row >= N || col0 + kBN > N ||
-                             win_cuts(q0, q0 + kBM - 1, col0, col0 + kBN - 1, p.wl, p.wr);
-      // this row's visible keys: [klo, khi] (empty past N)
-      const int klo = (p.wl >= 0) ? row - p.wl : 0;
-      const int khi = (row >= N) ? -1 : min(N - 1, (p.wr >= 0) ? row + p.wr : N - 1);
+      const int ent = ctl.tiles[j];
+      const int col0 = (ent & ~kFullBit) * kBN;
+      const bool need_mask = !(ent & kFullBit);
 #pragma unroll 1
       for (int ck = 0; ck < kBN / 32; ++ck) {
         uint32_t sv[32], dp[32];
@@ -326,20 +345,16 @@ cudaError_t launch(const Problem& pr) {
   kp.nb = pr.nb;
   kp.nqt = pr.nb;   // 128-row query tiles
   kp.causal = pr.causal;
-  // a bound of N or more cuts nothing: unbounded (keeps row +- bound in int range)
-  kp.wl = (pr.wl >= pr.N) ? -1 : pr.wl;
-  kp.wr = pr.causal ? 0 : ((pr.wr >= pr.N) ? -1 : pr.wr);   // causal is the window wr = 0
+  kp.mod = mask_mod_of(pr);
   kp.BH = (int)BHq;
   kp.grad_bf16 = pr.grad_dtype == 1;
   kp.c = pr.scale * kLog2e;
   kp.scale = pr.scale;
+  kp.stall = debug_stall_cycles(kStallDq);
   const size_t smem = sizeof(Ctl) + 1024 + C::kOffEnd;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  {
+    const cudaError_t e = set_max_dynamic_smem((const void*)dq_kernel<D>, (int)smem);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   dim3 grid((unsigned)(BHq * kp.nqt));
   dq_kernel<D><<<grid, kThreads, smem, pr.stream>>>(kp);

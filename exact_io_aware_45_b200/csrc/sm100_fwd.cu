@@ -48,6 +48,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "sm100_common.cuh"
 
@@ -64,14 +65,38 @@ constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kTau = 8.0f;       // reference-max slack, log2 units
 constexpr int kMaxChunk = 16;      // most heads interleaved in launch order
 
-template <int D>
+constexpr int kMaxSlots = 10;     // most K/V ring slots of any form
+
+// Build-time tuning (defaults measured on B200): K/V ring slots of the
+// lockstep form at d = 128, and the FMA-pipe share of the softmax
+// exponentials in eighths at d = 64 and d = 128.
+#ifndef FA_FWD_SLOTS_D128
+#define FA_FWD_SLOTS_D128 5
+#endif
+#ifndef FA_FWD_EMU_PAIRS_D64
+#define FA_FWD_EMU_PAIRS_D64 0
+#endif
+#ifndef FA_FWD_EMU_PAIRS_D128
+#define FA_FWD_EMU_PAIRS_D128 0
+#endif
+// 1: dense and causal launches run the persistent form (one CTA per SM).
+#ifndef FA_FWD_PERSIST
+#define FA_FWD_PERSIST 1
+#endif
+
+template <int D, bool kSkip>
 struct Cfg {
-  static constexpr int kStages = (D == 64) ? 4 : 2;
-  // Share of the softmax exponentials computed on the FMA pipe, in eighths.
-  // Measured on B200 (llama7b-shaped causal and 16K GQA workloads): 0 is
-  // fastest here (the MUFU unit is not this kernel's bottleneck), so the
-  // FMA-pipe path is compiled in but off.
-  static constexpr int kEmuPairs = 0;
+  // K and V tiles share one ring of slots, loaded in the order they are
+  // consumed (K_0, V_0, K_1, V_1, ...) and released one by one (K_j once the
+  // last S MMA that reads it has completed, V_j after the last P V), so the
+  // load of K_{j+3} can start while iteration j is still running. The
+  // lockstep form keeps no tile lists and spends that shared memory on more
+  // slots: 5 x 32 KB at d = 128 (plus 64 KB of Q: 224 KB).
+  static constexpr int kSlots =
+      kSkip ? ((D == 64) ? 8 : 4) : ((D == 64) ? 10 : FA_FWD_SLOTS_D128);
+  // Share of the softmax exponentials computed on the FMA pipe, in eighths
+  // (tiles without masked scores only).
+  static constexpr int kEmuPairs = (D == 64) ? FA_FWD_EMU_PAIRS_D64 : FA_FWD_EMU_PAIRS_D128;
   static constexpr int kTileBytes = kBN * D * 2;   // one K or V tile (bf16)
   static constexpr int kQBytes = kBM * D * 2;
   static constexpr int kColBlocks = D / 64;        // 128-byte column blocks per row
@@ -80,24 +105,49 @@ struct Cfg {
   static constexpr uint32_t kO0 = 256, kO1 = 256 + (D == 64 ? 64 : 128);
   static constexpr uint32_t kPOff = 64;            // P (bf16 pairs) inside S's columns
   static constexpr int kOffQ = 0;
-  static constexpr int kOffK = kOffQ + 2 * kQBytes;
-  static constexpr int kOffV = kOffK + kStages * kTileBytes;
-  static constexpr int kOffEnd = kOffV + kStages * kTileBytes;
+  static constexpr int kOffKV = kOffQ + 2 * kQBytes;
+  static constexpr int kOffEnd = kOffKV + kSlots * kTileBytes;
+  static_assert(kSlots <= kMaxSlots, "ring barriers");
 };
 
-struct alignas(16) Ctl {
+// Ring position of the n-th K/V tile loaded (K_j is n = 2j, V_j is n = 2j + 1).
+template <int kSlots>
+__device__ __forceinline__ int ring_slot(int n) { return n % kSlots; }
+template <int kSlots>
+__device__ __forceinline__ uint32_t ring_phase(int n) { return (n / kSlots) & 1; }
+
+struct alignas(16) CtlCore {
   uint64_t q_full;
-  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint64_t kv_full[kMaxSlots], kv_empty[kMaxSlots];
   uint64_t s_full[2], p_half[2], p_full[2];
   uint64_t o_ready[2];       // query tile t's last P V has completed (skipping form)
   uint64_t o_done;
+  uint64_t never;            // signalled by nothing (wait-limit test hook)
+  uint64_t qt_full[2], qt_empty[2];   // per query tile Q buffer (persistent form)
   uint32_t tmem_base;
   int abort;
+  int skip;                  // the error word was set at launch: the CTA does nothing
   int ntiles;
-  int nlive[2];                  // key tiles query tile t sees (skipping form)
+  int nlive[2];              // key tiles query tile t sees (skipping form)
+};
+
+// Key-tile lists of the skipping form. The lockstep form walks key tiles
+// 0 .. T-1 and needs none.
+struct TileLists {
   uint16_t tiles[kMaxTiles];
   uint8_t dead[kMaxTiles];       // bit t: query tile t sees nothing of this key tile
-  uint16_t seen[kMaxTiles][2];   // [n][t]: n-th key tile query tile t sees (skipping form)
+  uint16_t seen[kMaxTiles][2];   // [n][t]: n-th key tile query tile t sees, | kFullBit
+};
+
+// Flag on a list entry: every (query, key) pair of the tile is visible, so
+// its scores need no masking.
+constexpr uint16_t kFullBit = 0x8000;
+
+template <bool kSkip>
+struct Ctl : CtlCore {};
+template <>
+struct Ctl<true> : CtlCore {
+  TileLists l;
 };
 
 struct FwdParams {
@@ -107,11 +157,13 @@ struct FwdParams {
   const uint8_t* mask;
   unsigned* err;
   int N, Hq, Hkv, nb, nblk, causal, BH;
-  int wl, wr;                // visible keys: row - wl <= key <= row + wr (-1: unbounded)
+  MaskMod mod;               // keys each query sees (the causal flag is its wr = 0)
   float c;                   // scale * log2(e)
+  float cap1, cap2;          // soft-capping: scores in log2 units = cap1 * tanh(cap2 * q.k)
   const int* cu;             // variable-length batch: sequence offsets [B+1], or null
   int total;                 // packed rows (variable-length batch)
   int chunk;                 // heads interleaved in launch order
+  long long stall;           // > 0: injected wait of this many cycles (test hook)
 };
 
 // 32 pairs of scores -> p = 2^(s*c - mu) packed to bf16 pairs, with the
@@ -134,6 +186,116 @@ __device__ __forceinline__ void exp_pack32(const uint32_t* sr, float2 c2, float2
   }
 }
 
+// The online-softmax step of one key tile for this thread's row, after its
+// scores sr (already masked: -inf where not visible; in log2 units once
+// multiplied by c) have been loaded from TMEM: row maximum, a move of the
+// reference maximum m_ref when the tile's maximum exceeds it by more than
+// kTau (l and, for n > 0, the TMEM accumulator rescaled by
+// alpha = 2^(m_old - m_new)), p = 2^(s*c - m_ref) into the P columns of S
+// (half a row at a time: p_half after the first 64 keys so P V can start,
+// p_full after all of them) and l += rowsum p. n is the tile's index within
+// the item (no accumulator to rescale before the first).
+template <int D, int kEmuPairs>
+__device__ __forceinline__ void softmax_tile(uint32_t (&sr)[128], bool need_mask, float c, int n,
+                                             float& m_ref, float& l, uint32_t sreg,
+                                             uint32_t preg, uint32_t oreg, uint64_t* p_half,
+                                             uint64_t* p_full, int lane) {
+  // Row maximum: eight independent chains of three-input max.
+  float m8[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float* v = reinterpret_cast<const float*>(&sr[16 * k]);
+    float m = fmax3(v[0], v[1], v[2]);
+#pragma unroll
+    for (int i = 3; i < 15; i += 2) m = fmax3(m, v[i], v[i + 1]);
+    m8[k] = fmaxf(m, v[15]);
+  }
+  const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
+                         fmaxf(m8[6], m8[7]));
+  const float mx2 = mx * c;
+  const bool grow = mx2 > m_ref + kTau;
+  float alpha = 1.f;
+  if (grow) {
+    alpha = ex2(m_ref - mx2);   // 0 when there was no reference yet
+    m_ref = mx2;
+    l *= alpha;
+  }
+  const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
+  // p = 2^(s*c - mu), two lanes per FMA, four pair accumulators for the
+  // sum; P goes to TMEM half a row at a time to keep registers free. In
+  // tiles without masked scores a share of the exponentials (kEmuPairs of
+  // every 8 pairs) can run on the FMA pipe (exp2_poly2) instead of MUFU.
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+  const float2 c2 = make_float2(c, c), nmu2 = make_float2(-mu, -mu);
+  // The MMA warp starts P V on the first 64 keys as soon as their P is in
+  // TMEM (p_half), while this warpgroup computes the second half.
+#pragma unroll
+  for (int hf = 0; hf < 2; ++hf) {
+    uint32_t pk[32];
+    if (need_mask)
+      exp_pack32<false, kEmuPairs>(&sr[64 * hf], c2, nmu2, acc, pk);
+    else
+      exp_pack32<true, kEmuPairs>(&sr[64 * hf], c2, nmu2, acc, pk);
+    tmem_st32(preg + 32 * hf, pk);
+    if (hf == 0) {
+      // The accumulator holds P V of earlier tiles (complete: the commit
+      // that signalled S_t came after them); rescale it where the
+      // reference moved, before any P V of this tile is issued.
+      if (__any_sync(0xffffffffu, grow && n > 0)) {
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(oreg + cc * 32, o);
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+          tmem_st32(oreg + cc * 32, o);
+        }
+      }
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(p_half);
+    }
+  }
+  const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
+  l += (a01.x + a01.y) + (a23.x + a23.y);
+  tmem_st_wait();
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(p_full);
+}
+
+// Stores this thread's output row: O = acc / l (bf16, 16-byte vectors) from
+// the TMEM accumulator (or zeros when no P V ran into it) and LSE =
+// (m_ref + log2 l) ln 2 (-inf for a row with no visible key).
+template <int D>
+__device__ __forceinline__ void store_row(uint32_t oreg, bool have_o, float m_ref, float l,
+                                          bool valid, __nv_bfloat16* out, float* lse_out) {
+  const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    if (have_o) {
+      tmem_ld32(oreg + cc * 32, o);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = 0u;
+    }
+    uint4 v[4];
+    uint32_t* vw = reinterpret_cast<uint32_t*>(v);
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      vw[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
+#pragma unroll
+      for (int i = 0; i < 4; ++i) dst[i] = v[i];
+    }
+  }
+  if (valid) *lse_out = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+}
+
 // Bounded wait that ignores the abort flag (used only to drain in-flight work).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
@@ -142,13 +304,14 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-template <int D, bool kVarlen, bool kSkip>
+template <int D, bool kVarlen, bool kSkip, bool kCap>
 __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant__ FwdParams p) {
-  using C = Cfg<D>;
+  using C = Cfg<D, kSkip>;
+  constexpr int kSlots = C::kSlots;
   extern __shared__ uint8_t smem_raw[];
-  Ctl& ctl = *reinterpret_cast<Ctl*>(smem_raw);
+  Ctl<kSkip>& ctl = *reinterpret_cast<Ctl<kSkip>*>(smem_raw);
   const uint32_t raw_addr = smem_u32(smem_raw);
-  const uint32_t tile_addr = (raw_addr + sizeof(Ctl) + 1023u) & ~1023u;
+  const uint32_t tile_addr = (raw_addr + sizeof(Ctl<kSkip>) + 1023u) & ~1023u;
   uint8_t* tiles_base = smem_raw + (tile_addr - raw_addr);
 
   // Heads are taken p.chunk at a time (their K/V stay in L2 during a wave);
@@ -157,7 +320,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   chunked_order(blockIdx.x, p.nblk, p.BH, p.chunk, bh, rblk);
   // A launch whose error word is already set (an earlier wait ran out and
   // nobody has read the word yet) does no work: its inputs may be invalid.
-  if (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) return;
+  // One thread reads the word and the whole CTA leaves together, before any
+  // barrier is initialised or TMEM allocated (another CTA may set the word
+  // meanwhile, so per-thread reads could disagree).
+  if (threadIdx.x == 0) ctl.skip = (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) ? 1 : 0;
+  __syncthreads();
+  if (ctl.skip) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int blk = p.nblk - 1 - rblk;
   const int h = bh % p.Hq, b = bh / p.Hq;
@@ -178,12 +346,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     qplane = h;
     kplane = h / (p.Hq / p.Hkv);
   }
+  // Key tiles either query tile can see end before kb_end. The lockstep form
+  // runs without a block mask, a left window edge or documents, so every key
+  // tile below kb_end is seen by one of the two query tiles: its list is
+  // 0 .. kb_end-1 and needs no storage.
+  const int kb_end = min(nb, mod_last_key(p.mod, qb1 * kBM + kBM - 1, N) / kBN + 1);
 
   if (threadIdx.x == 0) {
     mbar_init(&ctl.q_full, 1);
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&ctl.k_full[s], 1);
-      mbar_init(&ctl.v_full[s], 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&ctl.kv_full[s], 1);
       mbar_init(&ctl.kv_empty[s], 1);
     }
     for (int t = 0; t < 2; ++t) {
@@ -193,50 +365,56 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       mbar_init(&ctl.o_ready[t], 1);
     }
     mbar_init(&ctl.o_done, 1);
+    mbar_init(&ctl.never, 1);
     ctl.abort = 0;
+    if constexpr (!kSkip) ctl.ntiles = kb_end;
     fence_mbar_init();
   }
   if (warp == 2) {
     tmem_alloc(&ctl.tmem_base, 512);
     tmem_relinquish();
   }
-  if (warp == 3) {
-    // Key tiles either query tile can see, in increasing order.
-    const int kb_end = p.wr >= 0 ? min(nb, (qb1 * kBM + kBM - 1 + p.wr) / kBN + 1) : nb;
-    int count = 0, live0 = 0, live1 = 0;
-    for (int kb0 = 0; kb0 < kb_end; kb0 += 32) {
-      const int kb = kb0 + lane;
-      bool a0 = false, a1 = false;
-      if (kb < kb_end) {
-        const int c0 = kb * kBN, c1 = c0 + kBN - 1;
-        a0 = (!p.mask || p.mask[(size_t)qb0 * p.nb + kb]) &&
-             win_any(qb0 * kBM, qb0 * kBM + kBM - 1, c0, c1, p.wl, p.wr);
-        a1 = qb1 < nb && (!p.mask || p.mask[(size_t)qb1 * p.nb + kb]) &&
-             win_any(qb1 * kBM, qb1 * kBM + kBM - 1, c0, c1, p.wl, p.wr);
-      }
-      const bool act = a0 || a1;
-      const unsigned bal = __ballot_sync(0xffffffffu, act);
-      if (act) {
-        const int pos = count + __popc(bal & ((1u << lane) - 1u));
-        ctl.tiles[pos] = static_cast<uint16_t>(kb);
-        ctl.dead[pos] = static_cast<uint8_t>((a0 ? 0 : 1) | (a1 ? 0 : 2));
-      }
-      if constexpr (kSkip) {
-        // and each query tile's own list
+  if constexpr (kSkip) {
+    if (warp == 3) {
+      // Key tiles either query tile can see, in increasing order, and each
+      // query tile's own list (entries flagged kFullBit need no masking).
+      int count = 0, live0 = 0, live1 = 0;
+      for (int kb0 = 0; kb0 < kb_end; kb0 += 32) {
+        const int kb = kb0 + lane;
+        int k0 = kTileEmpty, k1 = kTileEmpty;
+        if (kb < kb_end) {
+          const int c0 = kb * kBN, c1 = c0 + kBN - 1;
+          if (!p.mask || p.mask[(size_t)qb0 * p.nb + kb])
+            k0 = mod_classify(p.mod, qb0 * kBM, qb0 * kBM + kBM - 1, c0, c1, N);
+          if (qb1 < nb && (!p.mask || p.mask[(size_t)qb1 * p.nb + kb]))
+            k1 = mod_classify(p.mod, qb1 * kBM, qb1 * kBM + kBM - 1, c0, c1, N);
+        }
+        const bool a0 = k0 != kTileEmpty, a1 = k1 != kTileEmpty;
+        const bool act = a0 || a1;
         const unsigned below = (1u << lane) - 1u;
+        const unsigned bal = __ballot_sync(0xffffffffu, act);
+        if (act) {
+          const int pos = count + __popc(bal & below);
+          ctl.l.tiles[pos] = static_cast<uint16_t>(kb);
+          ctl.l.dead[pos] = static_cast<uint8_t>((a0 ? 0 : 1) | (a1 ? 0 : 2));
+        }
         const unsigned bal0 = __ballot_sync(0xffffffffu, a0);
         const unsigned bal1 = __ballot_sync(0xffffffffu, a1);
-        if (a0) ctl.seen[live0 + __popc(bal0 & below)][0] = static_cast<uint16_t>(kb);
-        if (a1) ctl.seen[live1 + __popc(bal1 & below)][1] = static_cast<uint16_t>(kb);
+        if (a0)
+          ctl.l.seen[live0 + __popc(bal0 & below)][0] =
+              static_cast<uint16_t>(kb | (k0 == kTileFull ? kFullBit : 0));
+        if (a1)
+          ctl.l.seen[live1 + __popc(bal1 & below)][1] =
+              static_cast<uint16_t>(kb | (k1 == kTileFull ? kFullBit : 0));
         live0 += __popc(bal0);
         live1 += __popc(bal1);
+        count += __popc(bal);
       }
-      count += __popc(bal);
-    }
-    if (lane == 0) {
-      ctl.ntiles = count;
-      ctl.nlive[0] = live0;
-      ctl.nlive[1] = live1;
+      if (lane == 0) {
+        ctl.ntiles = count;
+        ctl.nlive[0] = live0;
+        ctl.nlive[1] = live1;
+      }
     }
   }
   tc_fence_before();
@@ -245,6 +423,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   const uint32_t tm = ctl.tmem_base;
   const int T = ctl.ntiles;
   const Guard g{&ctl.abort, p.err};
+  // j-th key tile of the CTA's list
+  auto tile_of = [&](int j) -> int {
+    if constexpr (kSkip) return ctl.l.tiles[j];
+    else return j;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -257,28 +440,25 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         for (int cb = 0; cb < C::kColBlocks; ++cb)
           tma_load_3d(tiles_base + C::kOffQ + t * C::kQBytes + cb * C::kBlockBytes, &p.tq,
                       &ctl.q_full, cb * 64, row0 + q0 + t * kBM, qplane);
+      // K_0, V_0, K_1, V_1, ... into the slot ring, each slot reused once the
+      // MMA warp has released the tile kSlots loads earlier.
       int issued = 0;
-      for (int j = 0; j < T; ++j) {
-        const int s = j % C::kStages;
-        if (j >= C::kStages && !mbar_wait(&ctl.kv_empty[s], ((j / C::kStages) - 1) & 1, g))
-          break;
-        const int kb = ctl.tiles[j];
-        mbar_expect_tx(&ctl.k_full[s], C::kTileBytes);
+      for (int n = 0; n < 2 * T; ++n) {
+        const int s = ring_slot<kSlots>(n);
+        if (n >= kSlots && !mbar_wait(&ctl.kv_empty[s], ring_phase<kSlots>(n - kSlots), g)) break;
+        const int kb = tile_of(n >> 1);
+        const CUtensorMap* m = (n & 1) ? &p.tv : &p.tk;
+        mbar_expect_tx(&ctl.kv_full[s], C::kTileBytes);
         for (int cb = 0; cb < C::kColBlocks; ++cb)
-          tma_load_3d(tiles_base + C::kOffK + s * C::kTileBytes + cb * C::kBlockBytes, &p.tk,
-                      &ctl.k_full[s], cb * 64, row0 + kb * kBN, kplane);
-        mbar_expect_tx(&ctl.v_full[s], C::kTileBytes);
-        for (int cb = 0; cb < C::kColBlocks; ++cb)
-          tma_load_3d(tiles_base + C::kOffV + s * C::kTileBytes + cb * C::kBlockBytes, &p.tv,
-                      &ctl.v_full[s], cb * 64, row0 + kb * kBN, kplane);
-        issued = j + 1;
+          tma_load_3d(tiles_base + C::kOffKV + s * C::kTileBytes + cb * C::kBlockBytes, m,
+                      &ctl.kv_full[s], cb * 64, row0 + kb * kBN, kplane);
+        issued = n + 1;
       }
       // Every issued copy has landed before the CTA may exit.
       drain_wait(&ctl.q_full, 0);
-      for (int s = 0; s < C::kStages && s < issued; ++s) {
-        const int n_s = (issued - 1 - s) / C::kStages + 1;  // loads into stage s
-        drain_wait(&ctl.k_full[s], (n_s - 1) & 1);
-        drain_wait(&ctl.v_full[s], (n_s - 1) & 1);
+      for (int s = 0; s < kSlots && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / kSlots) * kSlots;   // last load into slot s
+        drain_wait(&ctl.kv_full[s], ring_phase<kSlots>(last));
       }
     }
   } else if (warp == 1) {
@@ -287,10 +467,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       constexpr uint32_t idS = idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t idO = idesc_bf16(kBM, D, false, true);
       const uint32_t qa = smem_u32(tiles_base + C::kOffQ);
-      const uint32_t ka = smem_u32(tiles_base + C::kOffK);
-      const uint32_t va = smem_u32(tiles_base + C::kOffV);
-      auto issue_s = [&](int t, int stage) {
-        const uint32_t qt = qa + t * C::kQBytes, kt = ka + stage * C::kTileBytes;
+      const uint32_t kva = smem_u32(tiles_base + C::kOffKV);
+      auto slot_addr = [&](int n) { return kva + ring_slot<kSlots>(n) * C::kTileBytes; };
+      auto wait_tile = [&](int n) {
+        return mbar_wait(&ctl.kv_full[ring_slot<kSlots>(n)], ring_phase<kSlots>(n), g);
+      };
+      auto release_tile = [&](int n) { mma_commit(&ctl.kv_empty[ring_slot<kSlots>(n)]); };
+      // S_t = Q_t K_j^T
+      auto issue_s = [&](int t, int j) {
+        const uint32_t qt = qa + t * C::kQBytes, kt = slot_addr(2 * j);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
@@ -298,9 +483,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                  sdesc_sw128(kt + off, 16, 1024), idS, kk > 0);
         }
       };
-      // P V over keys 64*hf .. 64*hf+63 of the tile.
-      auto issue_pv = [&](int t, int stage, bool acc, int hf) {
-        const uint32_t vt = va + stage * C::kTileBytes;
+      // O_t += P_t V_j over keys 64*hf .. 64*hf+63 of the tile.
+      auto issue_pv = [&](int t, int j, bool acc, int hf) {
+        const uint32_t vt = slot_addr(2 * j + 1);
         const uint32_t pt = tm + (t ? C::kS1 : C::kS0) + C::kPOff;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
@@ -318,8 +503,9 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         // no shared-memory load sits between a signal and the next issue.
         const int nl0 = ctl.nlive[0], nl1 = ctl.nlive[1];
         int n0 = 0, n1 = 0;
-        int live_next = T > 0 ? (~ctl.dead[0] & 3) : 0;
-        bool ok = mbar_wait(&ctl.q_full, 0, g) && mbar_wait(&ctl.k_full[0], 0, g);
+        int live_next = T > 0 ? (~ctl.l.dead[0] & 3) : 0;
+        bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait(&ctl.q_full, 0, g) &&
+                  wait_tile(0);
         if (ok) {
           tc_fence_after();
           if (live_next & 1) {
@@ -330,87 +516,87 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             issue_s(1, 0);
             mma_commit(&ctl.s_full[1]);
           }
+          release_tile(0);
         }
         for (int j = 0; ok && j < T; ++j) {
-          const int s = j % C::kStages;
-          const uint32_t ph = (j / C::kStages) & 1;
           const bool more = j + 1 < T;
-          const int s2 = (j + 1) % C::kStages;
           const int live_cur = live_next;
-          live_next = more ? (~ctl.dead[j + 1] & 3) : 0;
-          if (!(ok = mbar_wait(&ctl.v_full[s], ph, g))) break;
+          live_next = more ? (~ctl.l.dead[j + 1] & 3) : 0;
+          if (!(ok = wait_tile(2 * j + 1))) break;
           if (live_cur & 1) {
             if (!(ok = mbar_wait(&ctl.p_half[0], n0 & 1, g))) break;
             tc_fence_after();
-            issue_pv(0, s, n0 > 0, 0);
+            issue_pv(0, j, n0 > 0, 0);
             if (!(ok = mbar_wait(&ctl.p_full[0], n0 & 1, g))) break;
             tc_fence_after();
-            issue_pv(0, s, n0 > 0, 1);
+            issue_pv(0, j, n0 > 0, 1);
             if (++n0 == nl0) mma_commit(&ctl.o_ready[0]);
           }
           if (more) {
-            if (!(ok = mbar_wait(&ctl.k_full[s2], ((j + 1) / C::kStages) & 1, g))) break;
+            if (!(ok = wait_tile(2 * j + 2))) break;
             tc_fence_after();
             if (live_next & 1) {
-              issue_s(0, s2);
+              issue_s(0, j + 1);
               mma_commit(&ctl.s_full[0]);
             }
           }
           if (live_cur & 2) {
             if (!(ok = mbar_wait(&ctl.p_half[1], n1 & 1, g))) break;
             tc_fence_after();
-            issue_pv(1, s, n1 > 0, 0);
+            issue_pv(1, j, n1 > 0, 0);
             if (!(ok = mbar_wait(&ctl.p_full[1], n1 & 1, g))) break;
             tc_fence_after();
-            issue_pv(1, s, n1 > 0, 1);
+            issue_pv(1, j, n1 > 0, 1);
             if (++n1 == nl1) mma_commit(&ctl.o_ready[1]);
           }
-          mma_commit(&ctl.kv_empty[s]);
-          if (more && (live_next & 2)) {
-            issue_s(1, s2);
-            mma_commit(&ctl.s_full[1]);
+          release_tile(2 * j + 1);   // V_j
+          if (more) {
+            if (live_next & 2) {
+              issue_s(1, j + 1);
+              mma_commit(&ctl.s_full[1]);
+            }
+            release_tile(2 * j + 2);   // K_{j+1}
           }
         }
         // Every query tile's epilogue gets its signal, also after an abort.
         if (n0 != nl0 || nl0 == 0) mma_commit(&ctl.o_ready[0]);
         if (n1 != nl1 || nl1 == 0) mma_commit(&ctl.o_ready[1]);
       } else {
-        bool ok = mbar_wait(&ctl.q_full, 0, g) && mbar_wait(&ctl.k_full[0], 0, g);
+        bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait(&ctl.q_full, 0, g) &&
+                  wait_tile(0);
         if (ok) {
           tc_fence_after();
           issue_s(0, 0);
           mma_commit(&ctl.s_full[0]);
           issue_s(1, 0);
           mma_commit(&ctl.s_full[1]);
+          release_tile(0);
         }
         for (int j = 0; ok && j < T; ++j) {
-          const int s = j % C::kStages;
-          const uint32_t ph = (j / C::kStages) & 1;
-          if (!(ok = mbar_wait(&ctl.v_full[s], ph, g) && mbar_wait(&ctl.p_half[0], j & 1, g)))
-            break;
+          if (!(ok = wait_tile(2 * j + 1) && mbar_wait(&ctl.p_half[0], j & 1, g))) break;
           tc_fence_after();
-          issue_pv(0, s, j > 0, 0);
+          issue_pv(0, j, j > 0, 0);
           if (!(ok = mbar_wait(&ctl.p_full[0], j & 1, g))) break;
           tc_fence_after();
-          issue_pv(0, s, j > 0, 1);
+          issue_pv(0, j, j > 0, 1);
           const bool more = j + 1 < T;
-          const int s2 = (j + 1) % C::kStages;
           if (more) {
-            if (!(ok = mbar_wait(&ctl.k_full[s2], ((j + 1) / C::kStages) & 1, g))) break;
+            if (!(ok = wait_tile(2 * j + 2))) break;
             tc_fence_after();
-            issue_s(0, s2);
+            issue_s(0, j + 1);
             mma_commit(&ctl.s_full[0]);
           }
           if (!(ok = mbar_wait(&ctl.p_half[1], j & 1, g))) break;
           tc_fence_after();
-          issue_pv(1, s, j > 0, 0);
+          issue_pv(1, j, j > 0, 0);
           if (!(ok = mbar_wait(&ctl.p_full[1], j & 1, g))) break;
           tc_fence_after();
-          issue_pv(1, s, j > 0, 1);
-          mma_commit(&ctl.kv_empty[s]);
+          issue_pv(1, j, j > 0, 1);
+          release_tile(2 * j + 1);   // V_j
           if (more) {
-            issue_s(1, s2);
+            issue_s(1, j + 1);
             mma_commit(&ctl.s_full[1]);
+            release_tile(2 * j + 2);   // K_{j+1}
           }
         }
       }
@@ -426,9 +612,17 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t sreg = tm + (t ? C::kS1 : C::kS0) + lane_off;
     const uint32_t oreg = tm + (t ? C::kO1 : C::kO0) + lane_off;
-    const float c = p.c;
+    // With soft-capping the scores are transformed into log2 units before the
+    // softmax (score modifier first, then the mask), so the exponent scale is 1.
+    const float c = kCap ? 1.f : p.c;
     const int tile_row0 = q0 + t * kBM;
     float m_ref = -INFINITY, l = 0.f;
+    // Skipping form: the keys this row sees (before the block mask, which is
+    // per tile), looked up once (documents take binary searches). The
+    // lockstep form has no documents and no left edge: its bounds are cheap
+    // to recompute where a tile needs masking.
+    int row_lo = 0, row_hi = N - 1;
+    if constexpr (kSkip) mod_row_keys(p.mod, row, N, row_lo, row_hi);
     // Lockstep form: every tile of the list, n = it. Skipping form: only the
     // tiles this query tile sees, it = 2n + t walking entry [n][t] of its list.
     constexpr int kStep = kSkip ? 2 : 1;
@@ -440,83 +634,39 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld128(sreg, sr);
-      const int col0 = (kSkip ? (&ctl.seen[0][0])[it] : ctl.tiles[it]) * kBN;
-      const bool dead = !kSkip && ((ctl.dead[it] >> t) & 1);
-      const bool need_mask = dead || col0 + kBN > N ||
-                             win_cuts(tile_row0, tile_row0 + kBM - 1, col0, col0 + kBN - 1, p.wl, p.wr);
+      if constexpr (kCap) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          sr[i] = __float_as_uint(p.cap1 * tanh_ex2(__uint_as_float(sr[i]) * p.cap2));
+      }
+      int col0;
+      bool dead = false, need_mask;
+      if constexpr (kSkip) {
+        const int e = (&ctl.l.seen[0][0])[it];
+        col0 = (e & ~kFullBit) * kBN;
+        need_mask = !(e & kFullBit);
+      } else {
+        // lockstep: key tile it; this query tile may see none of it (the
+        // causal diagonal or a right window edge of the other tile, or a
+        // second tile past the end of the sequence)
+        col0 = it * kBN;
+        // (the classification of mod_classify without documents or a left
+        // edge, and keys past N masked whatever the rows)
+        const int wr = p.mod.wr, pre1 = p.mod.prefix - 1;
+        dead = (t == 1 && qb1 >= nb) || (wr >= 0 && col0 > max(tile_row0 + kBM - 1 + wr, pre1));
+        need_mask = dead || col0 + kBN > N || (wr >= 0 && col0 + kBN - 1 > max(tile_row0 + wr, pre1));
+      }
       if (need_mask) {
+        if constexpr (!kSkip) mod_row_keys(p.mod, row, N, row_lo, row_hi);
         // this row's visible columns of the tile: [lo, hi] relative to col0
-        int lo = (p.wl >= 0) ? row - p.wl - col0 : 0;
-        int hi = min(N - 1, (p.wr >= 0) ? row + p.wr : N - 1) - col0;
-        if (dead) hi = lo - 1;
+        const int lo = row_lo - col0;
+        const int hi = dead ? lo - 1 : row_hi - col0;
 #pragma unroll
         for (int i = 0; i < 128; ++i)
           if (i < lo || i > hi) sr[i] = __float_as_uint(-INFINITY);
       }
-      // Row maximum: eight independent chains of three-input max.
-      float m8[8];
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        const float* v = reinterpret_cast<const float*>(&sr[16 * k]);
-        float m = fmax3(v[0], v[1], v[2]);
-#pragma unroll
-        for (int i = 3; i < 15; i += 2) m = fmax3(m, v[i], v[i + 1]);
-        m8[k] = fmaxf(m, v[15]);
-      }
-      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]),
-                             fmaxf(m8[6], m8[7]));
-      const float mx2 = mx * c;
-      const bool grow = mx2 > m_ref + kTau;
-      float alpha = 1.f;
-      if (grow) {
-        alpha = ex2(m_ref - mx2);   // 0 when there was no reference yet
-        m_ref = mx2;
-        l *= alpha;
-      }
-      const float mu = (m_ref == -INFINITY) ? 0.f : m_ref;
-      // p = 2^(s*c - mu), two lanes per FMA, four pair accumulators for the
-      // sum; P goes to TMEM half a row at a time to keep registers free. In
-      // tiles without masked scores a share of the exponentials (kEmuPairs of
-      // every 8 pairs) can run on the FMA pipe (exp2_poly2) instead of MUFU.
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                       make_float2(0.f, 0.f)};
-      const float2 c2 = make_float2(c, c), nmu2 = make_float2(-mu, -mu);
-      // The MMA warp starts P V on the first 64 keys as soon as their P is in
-      // TMEM (p_half), while this warpgroup computes the second half.
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        uint32_t pk[32];
-        if (need_mask)
-          exp_pack32<false, C::kEmuPairs>(&sr[64 * hf], c2, nmu2, acc, pk);
-        else
-          exp_pack32<true, C::kEmuPairs>(&sr[64 * hf], c2, nmu2, acc, pk);
-        tmem_st32(sreg + C::kPOff + 32 * hf, pk);
-        if (hf == 0) {
-          // The accumulator holds P V of earlier tiles (complete: the commit
-          // that signalled S_t came after them); rescale it where the
-          // reference moved, before any P V of this tile is issued.
-          if (__any_sync(0xffffffffu, grow && n > 0)) {
-#pragma unroll
-            for (int cc = 0; cc < D / 32; ++cc) {
-              uint32_t o[32];
-              tmem_ld32(oreg + cc * 32, o);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-              tmem_st32(oreg + cc * 32, o);
-            }
-          }
-          tmem_st_wait();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&ctl.p_half[t]);
-        }
-      }
-      const float2 a01 = fadd2(acc[0], acc[1]), a23 = fadd2(acc[2], acc[3]);
-      l += (a01.x + a01.y) + (a23.x + a23.y);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&ctl.p_full[t]);
+      softmax_tile<D, C::kEmuPairs>(sr, need_mask, c, n, m_ref, l, sreg, sreg + C::kPOff, oreg,
+                                    &ctl.p_half[t], &ctl.p_full[t], lane);
     }
     // ------------------------------------------------------------ epilogue
     // The accumulator holds something only if some P V ran into it.
@@ -529,34 +679,13 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       mbar_wait(kSkip ? &ctl.o_ready[t] : &ctl.o_done, 0, g);
       tc_fence_after();
     }
-    const float inv = (l > 0.f) ? 1.f / l : 0.f;
     const bool valid = row < N;
     // O rows: [B][H][N][d] (dense) or [total][H][d] (variable-length)
     const size_t o_base = kVarlen ? ((size_t)row0 * p.Hq + h) * D : (size_t)bh * p.N * D;
     const size_t o_rs = kVarlen ? (size_t)p.Hq * D : (size_t)D;
     const size_t lse_base = kVarlen ? (size_t)h * p.total + row0 : (size_t)bh * p.N;
-    __nv_bfloat16* out = p.O + o_base + (size_t)(valid ? row : 0) * o_rs;
-#pragma unroll
-    for (int cc = 0; cc < D / 32; ++cc) {
-      uint32_t o[32];
-      if (have_o) {
-        tmem_ld32(oreg + cc * 32, o);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) o[i] = 0u;
-      }
-      uint4 v[4];
-      uint32_t* vw = reinterpret_cast<uint32_t*>(v);
-#pragma unroll
-      for (int i = 0; i < 16; ++i)
-        vw[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
-      if (valid) {
-        uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = v[i];
-      }
-    }
-    if (valid) p.LSE[lse_base + row] = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+    store_row<D>(oreg, have_o, m_ref, l, valid, p.O + o_base + (size_t)(valid ? row : 0) * o_rs,
+                 p.LSE + lse_base + (valid ? row : 0));
   }
 
   tc_fence_before();
@@ -567,9 +696,282 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   }
 }
 
+// Persistent form of the lockstep forward (dense and causal launches, no
+// mask, window left edge or documents): one CTA per SM walks a static list
+// of work items (a (batch, head) and a block of two 128-row query tiles, in
+// the launch order of the one-item form: groups of heads that share L2,
+// longest causal blocks first), item w = blockIdx.x + k * gridDim.x. What a
+// CTA of the one-item form pays once per item is overlapped here with the
+// previous item: the Q tile t of item k+1 is loaded as soon as the last S_t
+// of item k has read the old one (qt_empty[t]), the K/V slot ring runs on
+// across items, the next item's first S is issued right after the last P V
+// of the current one, and the epilogue of item k (O from TMEM to global
+// memory) runs while the MMA warp works on item k+1. Barrier phases count
+// tiles and items per CTA; the per-item softmax state starts afresh.
+template <int D, bool kCap>
+__global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_constant__ FwdParams p) {
+  using C = Cfg<D, false>;
+  constexpr int kSlots = C::kSlots;
+  extern __shared__ uint8_t smem_raw[];
+  Ctl<false>& ctl = *reinterpret_cast<Ctl<false>*>(smem_raw);
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t tile_addr = (raw_addr + sizeof(Ctl<false>) + 1023u) & ~1023u;
+  uint8_t* tiles_base = smem_raw + (tile_addr - raw_addr);
+  // A launch whose error word is already set does no work (see fwd_kernel).
+  if (threadIdx.x == 0) ctl.skip = (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) ? 1 : 0;
+  __syncthreads();
+  if (ctl.skip) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int W = p.BH * p.nblk;   // work items
+  const int N = p.N, nb = p.nb;
+
+  // item w -> (bh, first query row, number of key tiles, kv plane)
+  struct Item {
+    int bh, q0, T, kplane;
+  };
+  auto item_of = [&](int w) {
+    int bh, rblk;
+    chunked_order(w, p.nblk, p.BH, p.chunk, bh, rblk);
+    const int blk = p.nblk - 1 - rblk;
+    Item it;
+    it.bh = bh;
+    it.q0 = blk * 2 * kBM;
+    it.T = min(nb, mod_last_key(p.mod, (2 * blk + 1) * kBM + kBM - 1, N) / kBN + 1);
+    it.kplane = (bh / p.Hq) * p.Hkv + (bh % p.Hq) / (p.Hq / p.Hkv);
+    return it;
+  };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&ctl.kv_full[s], 1);
+      mbar_init(&ctl.kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctl.qt_full[t], 1);
+      mbar_init(&ctl.qt_empty[t], 1);
+      mbar_init(&ctl.s_full[t], 1);
+      mbar_init(&ctl.p_half[t], 4);
+      mbar_init(&ctl.p_full[t], 4);
+      mbar_init(&ctl.o_ready[t], 1);
+    }
+    mbar_init(&ctl.o_done, 1);
+    mbar_init(&ctl.never, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 2) {
+    tmem_alloc(&ctl.tmem_base, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = ctl.tmem_base;
+  const Guard g{&ctl.abort, p.err};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      prefetch_tmap(&p.tq);
+      prefetch_tmap(&p.tk);
+      prefetch_tmap(&p.tv);
+      int n = 0;              // K/V tiles loaded into the ring so far
+      int qi[2] = {0, 0};     // loads of each Q tile buffer so far
+      bool ok = true;
+      for (int w = blockIdx.x; ok && w < W; w += gridDim.x) {
+        const Item it = item_of(w);
+        // Q tile t of this item once the previous item's last S_t has read
+        // the buffer
+        for (int t = 0; ok && t < 2; ++t) {
+          if (qi[t] > 0 && !(ok = mbar_wait(&ctl.qt_empty[t], (qi[t] - 1) & 1, g))) break;
+          mbar_expect_tx(&ctl.qt_full[t], C::kQBytes);
+          for (int cb = 0; cb < C::kColBlocks; ++cb)
+            tma_load_3d(tiles_base + C::kOffQ + t * C::kQBytes + cb * C::kBlockBytes, &p.tq,
+                        &ctl.qt_full[t], cb * 64, it.q0 + t * kBM, it.bh);
+          ++qi[t];
+        }
+        for (int j = 0; ok && j < 2 * it.T; ++j, ++n) {
+          const int s = ring_slot<kSlots>(n);
+          if (n >= kSlots && !(ok = mbar_wait(&ctl.kv_empty[s], ring_phase<kSlots>(n - kSlots), g)))
+            break;
+          const CUtensorMap* m = (j & 1) ? &p.tv : &p.tk;
+          mbar_expect_tx(&ctl.kv_full[s], C::kTileBytes);
+          for (int cb = 0; cb < C::kColBlocks; ++cb)
+            tma_load_3d(tiles_base + C::kOffKV + s * C::kTileBytes + cb * C::kBlockBytes, m,
+                        &ctl.kv_full[s], cb * 64, (j >> 1) * kBN, it.kplane);
+        }
+      }
+      // Every issued copy has landed before the CTA may exit.
+      for (int t = 0; t < 2; ++t)
+        if (qi[t] > 0) drain_wait(&ctl.qt_full[t], (qi[t] - 1) & 1);
+      for (int s = 0; s < kSlots && s < n; ++s) {
+        const int last = s + ((n - 1 - s) / kSlots) * kSlots;
+        drain_wait(&ctl.kv_full[s], ring_phase<kSlots>(last));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idS = idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t idO = idesc_bf16(kBM, D, false, true);
+      const uint32_t qa = smem_u32(tiles_base + C::kOffQ);
+      const uint32_t kva = smem_u32(tiles_base + C::kOffKV);
+      auto slot_addr = [&](int n) { return kva + ring_slot<kSlots>(n) * C::kTileBytes; };
+      auto wait_tile = [&](int n) {
+        return mbar_wait(&ctl.kv_full[ring_slot<kSlots>(n)], ring_phase<kSlots>(n), g);
+      };
+      auto release_tile = [&](int n) { mma_commit(&ctl.kv_empty[ring_slot<kSlots>(n)]); };
+      // S_t = Q_t K^T with K the ring tile n
+      auto issue_s = [&](int t, int n) {
+        const uint32_t qt = qa + t * C::kQBytes, kt = slot_addr(n);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          mma_ss(tm + (t ? C::kS1 : C::kS0), sdesc_sw128(qt + off, 16, 1024),
+                 sdesc_sw128(kt + off, 16, 1024), idS, kk > 0);
+        }
+      };
+      // O_t += P_t V over keys 64*hf .. 64*hf+63 of the ring tile n (a V tile)
+      auto issue_pv = [&](int t, int n, bool acc, int hf) {
+        const uint32_t vt = slot_addr(n);
+        const uint32_t pt = tm + (t ? C::kS1 : C::kS0) + C::kPOff;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * hf + k4;
+          mma_ts(tm + (t ? C::kO1 : C::kO0), pt + kk * 8,
+                 sdesc_sw128(vt + kk * 16 * 128, C::kBlockBytes, 1024), idO, (acc || kk > 0));
+        }
+      };
+      bool ok = injected_stall(&ctl.never, p.stall, g);
+      int n = 0, nt = 0, k = 0;   // ring tiles, softmax tiles, items so far
+      for (int w = blockIdx.x; ok && w < W; w += gridDim.x, ++k) {
+        const Item it = item_of(w);
+        const int T = it.T;
+        // K_j is ring tile n + 2j, V_j is n + 2j + 1
+        for (int t = 0; t < 2; ++t) {
+          if (!(ok = mbar_wait(&ctl.qt_full[t], k & 1, g) && wait_tile(n))) break;
+          tc_fence_after();
+          issue_s(t, n);
+          mma_commit(&ctl.s_full[t]);
+          if (T == 1) mma_commit(&ctl.qt_empty[t]);
+        }
+        if (!ok) break;
+        release_tile(n);
+        for (int j = 0; ok && j < T; ++j) {
+          const uint32_t ph = (nt + j) & 1;
+          const bool more = j + 1 < T;
+          if (!(ok = wait_tile(n + 2 * j + 1) && mbar_wait(&ctl.p_half[0], ph, g))) break;
+          tc_fence_after();
+          issue_pv(0, n + 2 * j + 1, j > 0, 0);
+          if (!(ok = mbar_wait(&ctl.p_full[0], ph, g))) break;
+          tc_fence_after();
+          issue_pv(0, n + 2 * j + 1, j > 0, 1);
+          if (!more) mma_commit(&ctl.o_ready[0]);
+          if (more) {
+            if (!(ok = wait_tile(n + 2 * j + 2))) break;
+            tc_fence_after();
+            issue_s(0, n + 2 * j + 2);
+            mma_commit(&ctl.s_full[0]);
+            if (j + 2 == T) mma_commit(&ctl.qt_empty[0]);
+          }
+          if (!(ok = mbar_wait(&ctl.p_half[1], ph, g))) break;
+          tc_fence_after();
+          issue_pv(1, n + 2 * j + 1, j > 0, 0);
+          if (!(ok = mbar_wait(&ctl.p_full[1], ph, g))) break;
+          tc_fence_after();
+          issue_pv(1, n + 2 * j + 1, j > 0, 1);
+          if (!more) mma_commit(&ctl.o_ready[1]);
+          release_tile(n + 2 * j + 1);   // V_j
+          if (more) {
+            issue_s(1, n + 2 * j + 2);
+            mma_commit(&ctl.s_full[1]);
+            if (j + 2 == T) mma_commit(&ctl.qt_empty[1]);
+            release_tile(n + 2 * j + 2);   // K_{j+1}
+          }
+        }
+        n += 2 * T;
+        nt += T;
+      }
+      mma_commit(&ctl.o_done);
+      drain_wait(&ctl.o_done, 0);   // no MMA may still run when TMEM is freed
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int t = (warp - 4) >> 2;           // query tile of this warpgroup
+    const int wq = warp & 3;                 // TMEM lane quarter of this warp
+    const int r = wq * 32 + lane;            // row inside the tile
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t sreg = tm + (t ? C::kS1 : C::kS0) + lane_off;
+    const uint32_t oreg = tm + (t ? C::kO1 : C::kO0) + lane_off;
+    const float c = kCap ? 1.f : p.c;
+    bool ok = true;
+    int nt = 0, k = 0;
+    for (int w = blockIdx.x; ok && w < W; w += gridDim.x, ++k) {
+      const Item it = item_of(w);
+      const int tile_row0 = it.q0 + t * kBM;
+      const int row = tile_row0 + r;
+      const bool tile_live = tile_row0 < N;   // the second tile may lie past the end
+      float m_ref = -INFINITY, l = 0.f;
+      for (int j = 0; j < it.T; ++j) {
+        if (!(ok = mbar_wait(&ctl.s_full[t], (nt + j) & 1, g))) break;
+        tc_fence_after();
+        uint32_t sr[128];
+        tmem_ld128(sreg, sr);
+        if constexpr (kCap) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            sr[i] = __float_as_uint(p.cap1 * tanh_ex2(__uint_as_float(sr[i]) * p.cap2));
+        }
+        const int col0 = j * kBN;
+        // as in the lockstep form: this query tile may see none of key tile j
+        const int wr = p.mod.wr, pre1 = p.mod.prefix - 1;
+        const bool dead =
+            !tile_live || (wr >= 0 && col0 > max(tile_row0 + kBM - 1 + wr, pre1));
+        const bool need_mask =
+            dead || col0 + kBN > N || (wr >= 0 && col0 + kBN - 1 > max(tile_row0 + wr, pre1));
+        if (need_mask) {
+          int row_lo, row_hi;
+          mod_row_keys(p.mod, row, N, row_lo, row_hi);
+          const int lo = row_lo - col0;
+          const int hi = dead ? lo - 1 : row_hi - col0;
+#pragma unroll
+          for (int i = 0; i < 128; ++i)
+            if (i < lo || i > hi) sr[i] = __float_as_uint(-INFINITY);
+        }
+        softmax_tile<D, C::kEmuPairs>(sr, need_mask, c, j, m_ref, l, sreg, sreg + C::kPOff, oreg,
+                                      &ctl.p_half[t], &ctl.p_full[t], lane);
+      }
+      if (!ok) break;
+      nt += it.T;
+      // epilogue of this item: the last P V of this query tile has completed
+      if (!(ok = mbar_wait(&ctl.o_ready[t], k & 1, g))) break;
+      tc_fence_after();
+      const bool valid = row < N;
+      store_row<D>(oreg, true, m_ref, l, valid,
+                   p.O + ((size_t)it.bh * N + (valid ? row : 0)) * D,
+                   p.LSE + (size_t)it.bh * N + (valid ? row : 0));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tm, 512);
+  }
+}
+
+// Dynamic shared memory of one form: control block, alignment slack, tiles.
+template <int D, bool kSkip>
+constexpr size_t smem_bytes() {
+  return sizeof(Ctl<kSkip>) + 1024 + Cfg<D, kSkip>::kOffEnd;
+}
+static_assert(smem_bytes<128, false>() <= 232448 && smem_bytes<128, true>() <= 232448 &&
+                  smem_bytes<64, false>() <= 232448 && smem_bytes<64, true>() <= 232448,
+              "227 KB of shared memory per CTA");
+
 template <int D>
 cudaError_t launch(const Problem& pr) {
-  using C = Cfg<D>;
   FwdParams kp;
   memset(&kp, 0, sizeof(kp));
   const uint64_t BHq = (uint64_t)pr.B * pr.Hq;
@@ -589,23 +991,24 @@ cudaError_t launch(const Problem& pr) {
   kp.nb = pr.nb;
   kp.nblk = (pr.N + 2 * kBM - 1) / (2 * kBM);
   kp.causal = pr.causal;
-  // a bound of N or more cuts nothing: unbounded (keeps row +- bound in int range)
-  kp.wl = (pr.wl >= pr.N) ? -1 : pr.wl;
-  kp.wr = pr.causal ? 0 : ((pr.wr >= pr.N) ? -1 : pr.wr);   // causal is the window wr = 0
+  kp.mod = mask_mod_of(pr);
   kp.c = pr.scale * kLog2e;
+  const bool cap = pr.softcap > 0.f;
+  kp.cap1 = cap ? pr.softcap * kLog2e : 0.f;
+  kp.cap2 = cap ? pr.scale / pr.softcap : 0.f;
   kp.cu = pr.cu;
   kp.total = pr.total;
-  const size_t smem = sizeof(Ctl) + 1024 + C::kOffEnd;
-  static bool attr_set = false;
-  if (!attr_set) {
-    for (const void* f : {(const void*)fwd_kernel<D, false, false>,
-                          (const void*)fwd_kernel<D, false, true>,
-                          (const void*)fwd_kernel<D, true, false>}) {
-      const cudaError_t e =
-          cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e != cudaSuccess) return e;
-    }
-    attr_set = true;
+  kp.stall = debug_stall_cycles(kStallFwd);
+  const size_t smem_lock = smem_bytes<D, false>(), smem_skip = smem_bytes<D, true>();
+  for (const auto& fs : {std::make_pair((const void*)fwd_kernel<D, false, false, false>, smem_lock),
+                         std::make_pair((const void*)fwd_kernel<D, true, false, false>, smem_lock),
+                         std::make_pair((const void*)fwd_kernel<D, false, true, false>, smem_skip),
+                         std::make_pair((const void*)fwd_kernel<D, false, false, true>, smem_lock),
+                         std::make_pair((const void*)fwd_kernel<D, false, true, true>, smem_skip),
+                         std::make_pair((const void*)fwd_persist_kernel<D, false>, smem_lock),
+                         std::make_pair((const void*)fwd_persist_kernel<D, true>, smem_lock)}) {
+    const cudaError_t e = set_max_dynamic_smem(fs.first, (int)fs.second);
+    if (e != cudaSuccess) return e;
   }
   kp.BH = (int)BHq;
   // As many heads at a time as keep their K and V within about half of the
@@ -616,15 +1019,39 @@ cudaError_t launch(const Problem& pr) {
   const uint64_t per_kv = std::max<uint64_t>(1, (64ull << 20) / kv_bytes);
   kp.chunk = (int)std::min<uint64_t>(kMaxChunk, std::max<uint64_t>(1, per_kv) * (pr.Hq / pr.Hkv));
   dim3 grid((unsigned)(BHq * kp.nblk));
-  // Skip dead query-tile halves where they are common: block-sparse masks and
-  // windows with a left edge (variable-length batches take neither).
-  const bool skip = !pr.cu && (pr.mask != nullptr || kp.wl >= 0);
+  // Skip dead query-tile halves where they are common: block-sparse masks,
+  // windows with a left edge and documents (variable-length batches take
+  // none of them). The lockstep form walks key tiles 0 .. T-1 and relies on
+  // having none.
+  const bool gaps = pr.mask != nullptr || kp.mod.wl >= 0 || kp.mod.doc != nullptr;
+  const bool skip = !pr.cu && gaps;
+  if (!skip && gaps) return cudaErrorInvalidValue;
+  if (pr.cu && cap) return cudaErrorInvalidValue;   // not offered for packed batches
+  if (FA_FWD_PERSIST && !pr.cu && !skip) {
+    // one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
+    int dev = 0, sms = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t items = BHq * (uint64_t)kp.nblk;
+    const dim3 pgrid((unsigned)std::min<uint64_t>(items, (uint64_t)std::max(sms, 1)));
+    if (cap)
+      fwd_persist_kernel<D, true><<<pgrid, kThreads, smem_lock, pr.stream>>>(kp);
+    else
+      fwd_persist_kernel<D, false><<<pgrid, kThreads, smem_lock, pr.stream>>>(kp);
+    count_launch();
+    return cudaGetLastError();
+  }
   if (pr.cu)
-    fwd_kernel<D, true, false><<<grid, kThreads, smem, pr.stream>>>(kp);
+    fwd_kernel<D, true, false, false><<<grid, kThreads, smem_lock, pr.stream>>>(kp);
+  else if (skip && cap)
+    fwd_kernel<D, false, true, true><<<grid, kThreads, smem_skip, pr.stream>>>(kp);
   else if (skip)
-    fwd_kernel<D, false, true><<<grid, kThreads, smem, pr.stream>>>(kp);
+    fwd_kernel<D, false, true, false><<<grid, kThreads, smem_skip, pr.stream>>>(kp);
+  else if (cap)
+    fwd_kernel<D, false, false, true><<<grid, kThreads, smem_lock, pr.stream>>>(kp);
   else
-    fwd_kernel<D, false, false><<<grid, kThreads, smem, pr.stream>>>(kp);
+    fwd_kernel<D, false, false, false><<<grid, kThreads, smem_lock, pr.stream>>>(kp);
   count_launch();
   return cudaGetLastError();
 }

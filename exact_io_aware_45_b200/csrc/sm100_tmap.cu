@@ -1,9 +1,12 @@
-// Host-side construction of TMA tensor maps through the driver entry point
-// (no link-time dependency on libcuda).
+// Host-side helpers of the tcgen05 kernels: TMA tensor maps built through the
+// driver entry point (no link-time dependency on libcuda), and the per-device
+// shared-memory opt-in of the kernels.
 #include <cuda.h>
 #include <cuda_runtime.h>
 
 #include <mutex>
+#include <set>
+#include <tuple>
 
 #include "sm100_common.cuh"
 
@@ -60,6 +63,22 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int 
                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+cudaError_t set_max_dynamic_smem(const void* fn, int bytes) {
+  // The attribute belongs to the device that is current when it is set, so
+  // it is set once per (device, kernel, size); host threads share the record.
+  static std::mutex mu;
+  static std::set<std::tuple<int, const void*, int>> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const auto key = std::make_tuple(dev, fn, bytes);
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count(key)) return cudaSuccess;
+  e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.insert(key);
+  return e;
 }
 
 }  // namespace fa

@@ -22,13 +22,15 @@ LIB_PATH = os.environ.get("FA_LIBRARY") or os.path.join(PKG, "_lib", "libfa.so")
 FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
 FA_F32, FA_BF16 = 0, 1
 PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
+FA_STALL_FWD, FA_STALL_BWD, FA_STALL_DQ = 1, 2, 4
 
 # every symbol include/fa.h declares
 EXPORTS = ("fa_status_string", "fa_version", "fa_fwd_workspace_size", "fa_bwd_workspace_size",
            "fa_fwd", "fa_fwd_ex", "fa_bwd", "fa_bwd_ex", "fa_bwd_preprocess", "fa_bwd_main",
            "fa_bwd_finalize", "fa_last_launch_count", "fa_get_device_error", "fa_exp2_fma",
            "fa_fwd_varlen", "fa_bwd_varlen", "fa_bwd_varlen_workspace_size",
-           "fa_bwd_deterministic", "fa_fwd_window", "fa_bwd_window")
+           "fa_bwd_deterministic", "fa_fwd_window", "fa_bwd_window", "fa_bwd_noalloc",
+           "fa_debug_set_stall", "fa_fwd_mod", "fa_bwd_mod")
 
 _lib = None
 
@@ -39,6 +41,20 @@ _S = ctypes.c_size_t
 _FWD_ARGS = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _I, _P, _P]
 _BWD_ARGS = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P, _I, _I, _P, _S,
              _P]
+
+
+class FaMods(ctypes.Structure):
+    """fa_mods of include/fa.h: mask (and score) modifiers."""
+    _fields_ = [("window_left", ctypes.c_int), ("window_right", ctypes.c_int),
+                ("prefix", ctypes.c_int), ("doc_ids", ctypes.c_void_p),
+                ("softcap", ctypes.c_float)]
+
+
+def mods(window_left: int = -1, window_right: int = -1, prefix: int = 0, doc_ids=None,
+         softcap: float = 0.0) -> FaMods:
+    """An fa_mods value; doc_ids is an int32 CUDA tensor [N] or None."""
+    return FaMods(int(window_left), int(window_right), int(prefix),
+                  None if doc_ids is None else doc_ids.data_ptr(), float(softcap))
 
 
 class FaError(RuntimeError):
@@ -86,6 +102,14 @@ def lib() -> ctypes.CDLL:
         L.fa_bwd_window.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F,
                                     _I, _I, _I, _P, _I, _I, _P, _S, _P]
         L.fa_bwd_window.restype = _I
+        L.fa_fwd_mod.argtypes = [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P,
+                                 ctypes.POINTER(FaMods), _I, _P, _P]
+        L.fa_fwd_mod.restype = _I
+        L.fa_bwd_mod.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I,
+                                 _P, ctypes.POINTER(FaMods), _I, _I, _P, _S, _P]
+        L.fa_bwd_mod.restype = _I
+        L.fa_debug_set_stall.argtypes = [_I, ctypes.c_longlong]
+        L.fa_debug_set_stall.restype = _I
         L.fa_bwd_varlen_workspace_size.argtypes = [_I, _I, _I, _I, _I]
         L.fa_bwd_varlen_workspace_size.restype = _S
         _lib = L
@@ -168,6 +192,18 @@ def fa_fwd_varlen(*args) -> int:
 
 def fa_bwd_varlen(*args) -> int:
     return lib().fa_bwd_varlen(*args)
+
+
+def fa_fwd_mod(*args) -> int:
+    return lib().fa_fwd_mod(*args)
+
+
+def fa_bwd_mod(*args) -> int:
+    return lib().fa_bwd_mod(*args)
+
+
+def fa_debug_set_stall(kernels: int, wait_cycles: int) -> int:
+    return lib().fa_debug_set_stall(int(kernels), int(wait_cycles))
 
 
 def fa_bwd_varlen_workspace_size(B, Hq, max_seqlen, total, d) -> int:
@@ -336,6 +372,44 @@ def backward_window(q, k, v, o, do, lse, window_left: int, window_right: int,
                       int(window_left), int(window_right), _ptr(block_mask), _dtype_code(q.dtype),
                       _dtype_code(gdt), _ptr(ws), ws.numel(), _stream())
     _check(s, "fa_bwd_window")
+    return dq, dk, dv
+
+
+def forward_mod(q, k, v, m: FaMods, scale: Optional[float] = None, causal: bool = False,
+                block_mask=None, workspace=None):
+    """O, LSE with mask modifiers (fa_fwd_mod); layouts as forward."""
+    import torch
+    B, Hq, Hkv, N, d = _dims(q, k)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o = torch.empty_like(q)
+    l = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    ws = new_workspace(fa_fwd_workspace_size(), q.device) if workspace is None else workspace
+    s = fa_fwd_mod(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, float(scale),
+                   int(bool(causal)), _ptr(block_mask), ctypes.byref(m), _dtype_code(q.dtype),
+                   _ptr(ws), _stream())
+    _check(s, "fa_fwd_mod")
+    return o, l
+
+
+def backward_mod(q, k, v, o, do, lse, m: FaMods, scale: Optional[float] = None,
+                 causal: bool = False, block_mask=None, grad_dtype=None, workspace=None):
+    """dQ, dK, dV with mask modifiers (fa_bwd_mod); the forward's modifiers."""
+    import torch
+    B, Hq, Hkv, N, d = _dims(q, k)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    gdt = torch.float32 if grad_dtype is None else grad_dtype
+    dq = torch.empty(q.shape, dtype=gdt, device=q.device)
+    dk = torch.empty(k.shape, dtype=gdt, device=q.device)
+    dv = torch.empty(v.shape, dtype=gdt, device=q.device)
+    ws = new_workspace(fa_bwd_workspace_size(B, Hq, N, d), q.device) if workspace is None \
+        else workspace
+    s = fa_bwd_mod(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(do), _ptr(lse), _ptr(dq), _ptr(dk),
+                   _ptr(dv), B, Hq, Hkv, N, d, float(scale), int(bool(causal)), _ptr(block_mask),
+                   ctypes.byref(m), _dtype_code(q.dtype), _dtype_code(gdt), _ptr(ws), ws.numel(),
+                   _stream())
+    _check(s, "fa_bwd_mod")
     return dq, dk, dv
 
 

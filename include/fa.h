@@ -183,6 +183,57 @@ fa_status fa_bwd_window(const void* Q, const void* K, const void* V, const void*
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Mask and score modifiers: one tiled kernel, many masks (the lesson's
+ * Researcher section, "Beyond hand-written kernels", on FlexAttention's
+ * mask_mod and score_mod).
+ * With modifiers, key j is visible to query i iff lo(i) <= j <= hi(i) and the
+ * block mask allows the pair, where
+ *   hi(i) = min(right(i), last row of i's document),
+ *   lo(i) = max(window_left >= 0 ? i - window_left : 0, first row of i's document),
+ *   right(i) = N - 1 without a right bound, else max(i + r, prefix - 1) with
+ *   r = 0 under the causal flag (it wins over window_right), window_right
+ *   otherwise.
+ * Fields:
+ *   window_left, window_right: sliding-window bounds, -1 = unbounded;
+ *   prefix: >= 0; the first `prefix` keys are visible to every query whatever
+ *     the right bound says (with the causal flag: a prefix language model, the
+ *     prefix attending to itself in both directions);
+ *   doc_ids: NULL, or device int32 [N], 4-byte aligned, one document id per
+ *     token, non-decreasing (documents packed back to back; shared by every
+ *     batch and head): a query sees only keys of its own document. Ids that
+ *     are not sorted give wrong results but no access outside the array;
+ *   softcap: >= 0; 0 = off. A score modifier (FlexAttention's score_mod):
+ *     every score x = scale * q.k becomes softcap * tanh(x / softcap) before
+ *     the mask and the softmax; the backward applies the chain rule
+ *     d/dx = 1 - tanh^2(x / softcap). LSE is the logsumexp of the capped
+ *     scores. Not combined with variable-length batches.
+ * The backward must get the forward's modifiers. Tiles a query tile cannot
+ * see are skipped; tiles it sees whole run unmasked; the rest are masked per
+ * element. Tensor-core kernels only (dtype bf16, d in {64, 128}, scale > 0):
+ * FA_ERR_UNSUPPORTED otherwise; FA_ERR_INVALID_ARG for a bound below -1, a
+ * negative prefix, a misaligned doc_ids or a negative or non-finite softcap. mods == NULL, or all fields off,
+ * is fa_fwd / fa_bwd.
+ */
+typedef struct {
+  int window_left;
+  int window_right;
+  int prefix;
+  const int* doc_ids;
+  float softcap;
+} fa_mods;
+
+fa_status fa_fwd_mod(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                     int Hq, int Hkv, int N, int d, float scale, int causal,
+                     const uint8_t* block_mask, const fa_mods* mods, int dtype, void* workspace,
+                     void* stream);
+
+fa_status fa_bwd_mod(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                     const float* LSE, void* dQ, void* dK, void* dV, int B, int Hq, int Hkv,
+                     int N, int d, float scale, int causal, const uint8_t* block_mask,
+                     const fa_mods* mods, int dtype, int grad_dtype, void* workspace,
+                     size_t workspace_bytes, void* stream);
+
+/*
  * fa_bwd with run-to-run identical gradients. fa_bwd adds the dQ partials of
  * different key tiles with fp32 reduce-adds whose order depends on
  * scheduling, so its dQ can differ in the last bits between runs (dK, dV
@@ -256,7 +307,9 @@ size_t fa_bwd_varlen_workspace_size(int B, int Hq, int max_seqlen, int total, in
  * (FA_ERR_UNSUPPORTED otherwise, before anything is launched).
  * The first call on a device looks up the array's device address (with that
  * device current) and caches it; make that first call before any CUDA graph
- * capture. Every call on a device shares the one array and leaves its
+ * capture. The cached address is not looked up again, so fa_bwd_noalloc is
+ * not supported after cudaDeviceReset in the same process (the reset unloads
+ * the device image and the array may come back elsewhere). Every call on a device shares the one array and leaves its
  * contents behind; calls whose kernels overlap on the GPU (different streams
  * without ordering, or several host threads) race on it and must be ordered
  * by the caller.
@@ -280,6 +333,27 @@ fa_status fa_bwd_noalloc(const void* Q, const void* K, const void* V, const void
  * pointers with n > 0.
  */
 fa_status fa_exp2_fma(const float* x, float* y, long long n, void* stream);
+
+/*
+ * Test hook for the bounded-wait contract above ("Errors"); the pages have no
+ * counterpart. While on, every launch of the named tensor-core kernels makes
+ * its MMA-issuing thread wait first on an mbarrier that nothing ever
+ * signals, with a limit of wait_cycles SM clock cycles instead of the normal
+ * one of about 1.5 s. That wait runs out, the CTA sets FA_ERR_TIMEOUT's bit
+ * in the error word and takes the abort path (its other waits return at once,
+ * copies in flight are drained, TMEM is freed) and the kernel returns; CTAs
+ * that start after the word is set do nothing. The call's outputs are then
+ * undefined; nothing traps, faults or hangs, and after fa_get_device_error
+ * has cleared the word the workspace works normally again.
+ *   kernels: 0 (off) or an OR of FA_STALL_FWD (fa_fwd tensor-core kernel),
+ *            FA_STALL_BWD (backward main kernel), FA_STALL_DQ (the dQ kernel
+ *            of fa_bwd_deterministic);
+ *   wait_cycles: 1,000 .. 2,000,000,000 when kernels != 0 (ignored when 0).
+ * FA_ERR_INVALID_ARG otherwise. Process-wide (every host thread and device),
+ * read at each launch; for tests only.
+ */
+enum { FA_STALL_FWD = 1, FA_STALL_BWD = 2, FA_STALL_DQ = 4 };
+fa_status fa_debug_set_stall(int kernels, long long wait_cycles);
 
 /* Number of kernel launches the last successful call of fa_fwd_ex / fa_bwd_ex
  * or one of the stages made from the calling thread (for launch accounting). */

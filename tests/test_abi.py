@@ -118,3 +118,15 @@ def test_bwd_argument_checks(kw, want):
 
 def test_device_error_null_workspace():
     assert fa.fa_get_device_error(0, 0) == fa.FA_ERR_INVALID_ARG
+
+
+def test_debug_stall_hook_arguments():
+    """The wait-limit test hook validates its arguments and can be switched
+    off again (no kernel runs here)."""
+    assert fa.fa_debug_set_stall(0, 0) == fa.FA_OK
+    assert fa.fa_debug_set_stall(-1, 10_000) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_debug_set_stall(8, 10_000) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_debug_set_stall(fa.FA_STALL_FWD, 10) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_debug_set_stall(fa.FA_STALL_FWD, 3_000_000_000) == fa.FA_ERR_INVALID_ARG
+    assert fa.fa_debug_set_stall(fa.FA_STALL_FWD | fa.FA_STALL_DQ, 10_000) == fa.FA_OK
+    assert fa.fa_debug_set_stall(0, 0) == fa.FA_OK

@@ -195,6 +195,43 @@ def _sample_rows(rng, N, n):
     return np.unique(np.concatenate([[0, 1, 127, 128, N - 1], rng.choice(N, n, replace=False)]))
 
 
+# (batch, query head) pairs sampled at full size: first, last and interior heads
+QUERY_HEADS = {
+    "llama7b_causal": [(0, 0), (1, 7), (2, 19), (3, 31), (0, 16), (3, 1)],
+    "gqa16k_causal": [(0, 0), (0, 5), (0, 13), (0, 18), (0, 26), (0, 31)],
+    "sparse64k": [(0, 0), (0, 3), (0, 7), (0, 9), (0, 12), (0, 15)],
+}
+# (batch, KV head) pairs whose dK / dV rows are compared; for the grouped
+# workload every KV head collects the gradients of its 4 query heads, which
+# the oracle sums over the group
+KV_HEADS = {
+    "llama7b_causal": [(0, 0), (2, 13), (3, 31)],
+    "gqa16k_causal": [(0, 0), (0, 7)],
+    "sparse64k": [(0, 0), (0, 9)],
+}
+
+
+def _key_rows(rng, w, mask):
+    """Key rows whose dK / dV are compared at full size.
+
+    Causal workloads: key tile 0 (key 0 sees every query, so its dK / dV sum
+    the longest accumulation and hold the largest values), a tile in the
+    middle of the sequence and the last one. Block-sparse: block column 3 and
+    the block column with the most active cells."""
+    N = w.N
+    if w.causal:
+        mid = (N // 2 // 128) * 128
+        parts = [[0, 1, 127], rng.choice(128, 21, replace=False),
+                 [mid, mid + 127], mid + rng.choice(128, 14, replace=False),
+                 [N - 1], rng.choice(np.arange(N - 128, N), 12, replace=False)]
+    else:
+        dense_col = int(np.argmax(mask.sum(axis=0)))
+        parts = []
+        for kb in sorted({3, dense_col}):
+            parts += [[kb * 128, kb * 128 + 127], kb * 128 + rng.choice(128, 20, replace=False)]
+    return np.unique(np.concatenate([np.asarray(p, dtype=np.int64) for p in parts]))
+
+
 @pytest.mark.parametrize("name", ["gpt2_small", "llama7b_causal", "gqa16k_causal", "sparse64k"])
 def test_workload_parity(name):
     w = inputs.WORKLOADS[name]
@@ -216,9 +253,8 @@ def test_workload_parity(name):
         assert_close_bf16("dK", to_np(r["dk"]), dK)
         assert_close_bf16("dV", to_np(r["dv"]), dV)
         return
-    heads = [(0, 0), (w.B - 1, w.Hq - 1)]
     got_o, want_o, got_q, want_q = [], [], [], []
-    for b, h in heads:
+    for b, h in QUERY_HEADS[name]:
         rows = _sample_rows(rng, w.N, 96)
         Orow, Lrow = orc.forward_rows(x["q"], x["k"], x["v"], w.scale, w.causal, mask, b, h, rows)
         got_o.append(to_np(o[b, h, rows]))
@@ -229,23 +265,35 @@ def test_workload_parity(name):
                                   rows))
     assert_close_bf16("O rows", np.concatenate(got_o), np.concatenate(want_o))
     assert_close_bf16("dQ rows", np.concatenate(got_q), np.concatenate(want_q))
-    # key rows whose visible query set is bounded: for causal workloads keys in
-    # the last eighth of the sequence; for the block mask one key block
-    N = w.N
-    if w.causal:
-        keys = np.unique(np.concatenate([[N - 1], rng.choice(np.arange(N - N // 8, N), 48,
-                                                             replace=False)]))
-    else:
-        kb = 3
-        keys = np.unique(np.concatenate([[kb * 128, kb * 128 + 127],
-                                         rng.choice(np.arange(kb * 128, kb * 128 + 128), 30,
-                                                    replace=False)]))
-    got_k, want_k, got_v, want_v = [], [], [], []
-    for b, hk in [(0, 0), (w.B - 1, w.Hkv - 1)]:
-        dk, dv = orc.dkdv_rows(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal, mask, b, hk, keys)
-        got_k.append(to_np(r["dk"][b, hk, keys]))
-        want_k.append(dk)
-        got_v.append(to_np(r["dv"][b, hk, keys]))
-        want_v.append(dv)
-    assert_close_bf16("dK rows", np.concatenate(got_k), np.concatenate(want_k))
-    assert_close_bf16("dV rows", np.concatenate(got_v), np.concatenate(want_v))
+    keys = _key_rows(rng, w, mask)
+    for b, hk in KV_HEADS[name]:
+        dk, dv = orc.dkdv_rows(x["q"], x["k"], x["v"], x["do"], w.scale, w.causal, mask, b, hk,
+                               keys)
+        # each KV head on its own, so a wrong head or group sum cannot hide
+        # behind the others
+        assert_close_bf16(f"dK rows (b={b}, kv head {hk})", to_np(r["dk"][b, hk, keys]), dk)
+        assert_close_bf16(f"dV rows (b={b}, kv head {hk})", to_np(r["dv"][b, hk, keys]), dv)
+
+
+@pytest.mark.parametrize("dt_name", ["bf16", "f32"])
+def test_autograd_attention(dt_name):
+    """fa.attention through torch autograd: O from the forward, and the
+    gradients of sum(O * dO) (returned in the input dtype) against the oracle."""
+    import torch
+    dt = torch.bfloat16 if dt_name == "bf16" else torch.float32
+    x = inputs.random_case(1, 4, 2, 300, 64, seed=17, dtype=dt_name)
+    q, k, v = (to_dev(x[n], dt).requires_grad_(True) for n in ("q", "k", "v"))
+    do = to_dev(x["do"], dt)
+    scale = 0.125
+    o = fa.attention(q, k, v, scale, causal=True)
+    (o.float() * do.float()).sum().backward()
+    torch.cuda.synchronize()
+    O, _ = orc.forward(x["q"], x["k"], x["v"], scale, True)
+    dQ, dK, dV = orc.backward(x["q"], x["k"], x["v"], x["do"], scale, True, O=O)
+    for name, got, want in (("O", o, O), ("dQ", q.grad, dQ), ("dK", k.grad, dK),
+                            ("dV", v.grad, dV)):
+        assert got.dtype == dt
+        if dt_name == "bf16":
+            assert_close_bf16(name, to_np(got), want)
+        else:
+            assert max_abs(to_np(got), want) <= 1e-4, name

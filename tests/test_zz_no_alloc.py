@@ -24,15 +24,18 @@ def _noalloc_fn():
 
 
 @pytest.mark.parametrize("case", [
-    # B, Hq, Hkv, N, d, causal, mask density
-    (2, 4, 2, 300, 64, True, None),
-    (1, 2, 1, 640, 128, False, 0.5),
+    # B, Hq, Hkv, N, d, causal, mask density, input dtype
+    (2, 4, 2, 300, 64, True, None, "bf16"),      # tensor-core kernels
+    (1, 2, 1, 640, 128, False, 0.5, "bf16"),     # tensor-core kernels, block mask
+    (1, 2, 1, 200, 32, True, None, "f32"),       # CUDA-core kernels, fp32 inputs
+    (1, 4, 2, 257, 32, False, 0.5, "bf16"),      # CUDA-core kernels (d = 32), bf16 inputs
 ])
 def test_bwd_noalloc_matches_fa_bwd(case):
     import torch
-    B, Hq, Hkv, N, d, causal, dens = case
-    x = inputs.random_case(B, Hq, Hkv, N, d, seed=21 + N, mask_density=dens)
-    q, k, v, do = (to_dev(x[n], torch.bfloat16) for n in ("q", "k", "v", "do"))
+    B, Hq, Hkv, N, d, causal, dens, dt_name = case
+    dt = torch.bfloat16 if dt_name == "bf16" else torch.float32
+    x = inputs.random_case(B, Hq, Hkv, N, d, seed=21 + N, mask_density=dens, dtype=dt_name)
+    q, k, v, do = (to_dev(x[n], dt) for n in ("q", "k", "v", "do"))
     mask = None if x["mask"] is None else torch.from_numpy(x["mask"]).cuda()
     scale = 1.0 / np.sqrt(d)
     o, lse = fa.forward(q, k, v, scale, causal, mask)
@@ -47,7 +50,7 @@ def test_bwd_noalloc_matches_fa_bwd(case):
         dk = torch.full(k.shape, float("nan"), dtype=torch.float32, device="cuda")
         dv = torch.full(v.shape, float("nan"), dtype=torch.float32, device="cuda")
         s = f(P(q), P(k), P(v), P(o), P(do), P(lse), P(dq), P(dk), P(dv), B, Hq, Hkv, N, d,
-              float(scale), int(causal), P(mask), fa.FA_BF16,
+              float(scale), int(causal), P(mask), fa.FA_BF16 if dt_name == "bf16" else fa.FA_F32,
               P(err_word) if call == 0 else 0, stream)
         assert s == fa.FA_OK, fa.status_string(s)
         torch.cuda.synchronize()
