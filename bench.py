@@ -79,7 +79,7 @@ def workload_config(w: inputs.Workload, world: int, deterministic: bool = False,
             "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
             "block_sparse": w.sparse, "grad_dtype": "f32", "deterministic_dq": deterministic,
             "window_left": window,
-            "parallelism": f"replicas x{world} (independent batches)",
+            "parallelism": f"dp{world}: rank r owns global batch rows [rB, rB+B), all KV heads",
             "l2": "no flush: each of Q, K, V, dO is larger than L2 (126 MB)"
                   if w.B * w.Hq * w.N * w.d * 2 > 126e6 else "working set may fit L2"}
 
@@ -88,7 +88,7 @@ def forward_only_config(w: inputs.Workload, world: int) -> dict:
     return {"workload": f"{w.name}: B={w.B} H={w.Hq} N={w.N} d={w.d} "
                         f"{'causal' if w.causal else 'non-causal'} {w.dtype} forward",
             "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "causal": w.causal,
-            "block_sparse": w.sparse, "parallelism": f"replicas x{world} (independent batches)",
+            "block_sparse": w.sparse, "parallelism": f"dp{world}: rank r owns global batch rows [rB, rB+B), all KV heads",
             "l2": "flushed before every timed launch (a 256 MB write; inputs are 64 KB each)"}
 
 
@@ -240,6 +240,19 @@ def max_over_ranks(ms: float, device=None) -> float:
     t = torch.tensor([ms], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_units(world: int, rank: int, B: int, Hkv: int) -> list:
+    """The (global batch row, KV head) units rank ``rank`` owns. The units of
+    attention are independent (no exchange step on the pages' path), so the
+    job is partitioned, not replicated: the global problem holds ``world``
+    times the per-rank batch, and rank r owns batch rows r*B .. r*B + B - 1
+    with every KV head (each unit brings its group of query heads). Per-GPU
+    work stays fixed as ranks are added (weak scaling) and no collective
+    touches the data; rank r's rows are drawn with seed r."""
+    if not (0 <= rank < world):
+        raise ValueError("rank outside the job")
+    return [(rank * B + b, hk) for b in range(B) for hk in range(Hkv)]
 
 
 def job_tflops(flops_per_rank_step: float, steps: int, world: int, ms: float) -> float:

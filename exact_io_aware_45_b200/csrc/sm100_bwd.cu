@@ -59,7 +59,13 @@ constexpr int kChunk = FA_BWD_CHUNK;
 // 1: at d = 128 the two softmax warpgroups take alternate items (build-time
 // choice for A/B measurements; 0: one warpgroup takes every item).
 #ifndef FA_BWD_ITEM_SPLIT
-#define FA_BWD_ITEM_SPLIT 1
+#define FA_BWD_ITEM_SPLIT 0
+#endif
+// 1: at d = 128 the dQ drain adds into the fp32 accumulator with red.global
+// from registers instead of staging in shared memory for TMA reduce-adds
+// (build-time choice for A/B measurements).
+#ifndef FA_BWD_DQ_RED
+#define FA_BWD_DQ_RED 0
 #endif
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -101,6 +107,9 @@ struct Cfg {
   static constexpr int kOffVec = kOffStg + kStgBoxes * kStgBox;   // [stage][LSE2 | D][MQ]
   static constexpr int kOffEnd = kOffVec + kStages * 2 * MQ * 4;
   static_assert((kDbl ? kDP1 + MQ : kDQ + 64) <= 512, "TMEM budget");
+  // the dK / dV epilogue stages both fp32 tensors over the Q/dO ring and the
+  // dS buffers, which lie back to back before the dQ staging
+  static_assert(kOffStg - kOffQ >= 2 * kBN * D * 4, "epilogue staging");
 };
 
 struct alignas(16) Ctl {
@@ -123,8 +132,10 @@ struct BwdParams {
   CUtensorMap tq, tdo;         // [B*Hq][N][d] bf16, box {64, MQ}, 128B swizzle
   CUtensorMap tk, tv;          // [B*Hkv][N][d] bf16, box {64, 128}
   CUtensorMap tdq;             // [B*Hq][N][d] fp32, box {32, MQ}, 128B swizzle (reduce-add)
+  CUtensorMap tdk, tdv;        // [B*Hkv][N][d] grad dtype, box {128 bytes, 128}, 128B swizzle
   const float* lse2;           // [B*Hq][Npad]
   const float* dvec;           // [B*Hq][Npad]
+  float* dqacc;                // the fp32 dQ accumulator (layout of tdq)
   void* dK;
   void* dV;
   const uint8_t* mask;
@@ -163,13 +174,6 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   // under the causal flag, start first.
   int bhk, kb;
   chunked_order(blockIdx.x, p.nb, p.BHk, kChunk, bhk, kb);
-  // A launch whose error word is already set (an earlier wait ran out and
-  // nobody has read the word yet) does no work: its inputs may be invalid.
-  // One thread reads the word and the whole CTA leaves together, before any
-  // barrier is initialised or TMEM allocated.
-  if (threadIdx.x == 0) ctl.skip = (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) ? 1 : 0;
-  __syncthreads();
-  if (ctl.skip) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int n0 = kb * kBN;
   const int b = bhk / p.Hkv, hk = bhk % p.Hkv;
@@ -188,6 +192,12 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   const int kplane = kVarlen ? hk : bhk;
 
   if (threadIdx.x == 0) {
+    // A launch whose error word is already set (an earlier wait ran out and
+    // nobody has read the word yet) does no work: its inputs may be invalid.
+    // This one thread reads the word (while it sets up the barriers) and the
+    // whole CTA leaves together after the block barrier below, before any
+    // wait.
+    const unsigned err_word = *reinterpret_cast<volatile unsigned*>(p.err);
     mbar_init(&ctl.kv_full, 1);
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&ctl.qdo_full[s], 1);
@@ -203,6 +213,21 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
     mbar_init(&ctl.never, 1);
     ctl.abort = 0;
     fence_mbar_init();
+    ctl.skip = err_word != 0u;
+    if (!ctl.skip) {
+      // This thread is also the TMA producer: the K and V tiles start now, so
+      // their latency overlaps the TMEM allocation, the query-tile list and
+      // the block barrier.
+      prefetch_tmap(&p.tk);
+      prefetch_tmap(&p.tv);
+      mbar_expect_tx(&ctl.kv_full, 2 * C::kKVBytes);
+      for (int cb = 0; cb < D / 64; ++cb) {
+        tma_load_3d(base + C::kOffK + cb * kBN * 128, &p.tk, &ctl.kv_full, cb * 64, row0 + n0,
+                    kplane);
+        tma_load_3d(base + C::kOffV + cb * kBN * 128, &p.tv, &ctl.kv_full, cb * 64, row0 + n0,
+                    kplane);
+      }
+    }
   }
   if (warp == 2) {
     tmem_alloc(&ctl.tmem_base, 512);
@@ -233,6 +258,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = ctl.tmem_base;
+  if (ctl.skip) {   // the error word was set at launch: nothing was issued
+    if (warp == 2) tmem_dealloc(tm, 512);
+    return;
+  }
   const int nq = ctl.nq;
   const int n_items = nq * grp;
   const Guard g{&ctl.abort, p.err};
@@ -250,18 +279,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_items > 0) {
+    if (lane == 0) {
+      // (K and V were issued before the block barrier.)
       prefetch_tmap(&p.tq);
       prefetch_tmap(&p.tdo);
-      prefetch_tmap(&p.tk);
-      prefetch_tmap(&p.tv);
-      mbar_expect_tx(&ctl.kv_full, 2 * C::kKVBytes);
-      for (int cb = 0; cb < D / 64; ++cb) {
-        tma_load_3d(base + C::kOffK + cb * kBN * 128, &p.tk, &ctl.kv_full, cb * 64, row0 + n0,
-                    kplane);
-        tma_load_3d(base + C::kOffV + cb * kBN * 128, &p.tv, &ctl.kv_full, cb * 64, row0 + n0,
-                    kplane);
-      }
       int issued = 0;
       for (int i = 0; i < n_items; ++i) {
         const int s = i % C::kStages;
@@ -522,42 +543,105 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       tc_fence_after();
     }
     const bool valid = kv < N;
-    // dK, dV rows: [B][Hkv][N][d] (dense) or [total][Hkv][d] (variable-length)
-    const size_t orow = kVarlen ? ((size_t)(row0 + (valid ? kv : 0)) * p.Hkv + hk) * D
-                                : ((size_t)bhk * N + (valid ? kv : 0)) * D;
     // 8 softmax warps: warps 4-7 store dK, warps 8-11 dV; 4: warps 4-7 both.
+    const int which_lo = (C::kSoftWarps == 8) ? half : 0;
+    const int which_hi = (C::kSoftWarps == 8) ? half + 1 : 2;
+    if constexpr (!kVarlen) {
+      // dK and dV through the shared memory of the Q/dO ring and the dS
+      // buffers (every MMA has completed), in the TMA's 128-byte-swizzled
+      // layout: box b (128 bytes of each row: 32 fp32 or 64 bf16 columns) at
+      // b * 16 KB, row r at r * 128 bytes, 16-byte chunk c at ((c ^ (r & 7))
+      // << 4); dK first, dV after it. One thread then stores whole lines with
+      // TMA (rows at or past N are clipped by the tensor map).
+      const int esz = p.grad_bf16 ? 2 : 4;
+      const int tbytes = kBN * D * esz;   // one staged tensor
 #pragma unroll 1
-    for (int which = (C::kSoftWarps == 8) ? half : 0;
-         which < ((C::kSoftWarps == 8) ? half + 1 : 2); ++which) {
-      const uint32_t col = which ? C::kDV : C::kDK;
-      const float mul = which ? 1.f : p.scale;
+      for (int which = which_lo; which < which_hi; ++which) {
+        const uint32_t col = which ? C::kDV : C::kDK;
+        const float mul = which ? 1.f : p.scale;
+        uint8_t* st = base + C::kOffQ + which * tbytes;
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t v[32];
-        if (n_items > 0) {
-          tmem_ld32(tm + col + lane_off + cc * 32, v);
-        } else {
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t v[32];
+          if (n_items > 0) {
+            tmem_ld32(tm + col + lane_off + cc * 32, v);
+          } else {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = 0u;
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          if (p.grad_bf16) {
+            // 32 columns = 64 bytes: chunks 4 (cc & 1) .. +3 of box cc / 2
+            uint32_t w[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              w[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+            uint8_t* rowp = st + (cc >> 1) * 16384 + r * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int c = 4 * (cc & 1) + q;
+              *reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4)) =
+                  make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+            }
+          } else {
+            // 32 columns = 128 bytes: all 8 chunks of box cc
+            uint8_t* rowp = st + cc * 16384 + r * 128;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<float4*>(rowp + ((c ^ (r & 7)) << 4)) =
+                  make_float4(__uint_as_float(v[4 * c]) * mul, __uint_as_float(v[4 * c + 1]) * mul,
+                              __uint_as_float(v[4 * c + 2]) * mul,
+                              __uint_as_float(v[4 * c + 3]) * mul);
+          }
         }
-        if (!valid) continue;
-        if (p.grad_bf16) {
-          __nv_bfloat16* out = static_cast<__nv_bfloat16*>(which ? p.dV : p.dK) + orow + cc * 32;
-          uint32_t w[16];
+      }
+      fence_async_smem();
+      named_sync(2, C::kSoftWarps * 32);
+      if (warp == 4 && lane == 0) {
+        const int boxes = D * esz / 128, box_cols = 128 / esz;
+        for (int which = 0; which < 2; ++which)
+          for (int bx = 0; bx < boxes; ++bx)
+            tma_store_3d(which ? &p.tdv : &p.tdk, base + C::kOffQ + which * tbytes + bx * 16384,
+                         bx * box_cols, n0, bhk);
+        bulk_commit();
+        bulk_wait_read0();   // the staging is read before the CTA exits
+      }
+    } else {
+      // packed batch: a 128-row box could reach into the next sequence, so
+      // rows are stored one by one ([total][Hkv][d])
+      const size_t orow = ((size_t)(row0 + (valid ? kv : 0)) * p.Hkv + hk) * D;
+#pragma unroll 1
+      for (int which = which_lo; which < which_hi; ++which) {
+        const uint32_t col = which ? C::kDV : C::kDK;
+        const float mul = which ? 1.f : p.scale;
+#pragma unroll 1
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t v[32];
+          if (n_items > 0) {
+            tmem_ld32(tm + col + lane_off + cc * 32, v);
+          } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e)
-            w[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+            for (int e = 0; e < 32; ++e) v[e] = 0u;
+          }
+          if (!valid) continue;
+          if (p.grad_bf16) {
+            __nv_bfloat16* out = static_cast<__nv_bfloat16*>(which ? p.dV : p.dK) + orow + cc * 32;
+            uint32_t w[16];
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            reinterpret_cast<uint4*>(out)[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2],
-                                                          w[4 * e + 3]);
-        } else {
-          float* out = static_cast<float*>(which ? p.dV : p.dK) + orow + cc * 32;
+            for (int e = 0; e < 16; ++e)
+              w[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            reinterpret_cast<float4*>(out)[e] =
-                make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
-                            __uint_as_float(v[4 * e + 2]) * mul, __uint_as_float(v[4 * e + 3]) * mul);
+            for (int e = 0; e < 4; ++e)
+              reinterpret_cast<uint4*>(out)[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2],
+                                                            w[4 * e + 3]);
+          } else {
+            float* out = static_cast<float*>(which ? p.dV : p.dK) + orow + cc * 32;
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              reinterpret_cast<float4*>(out)[e] =
+                  make_float4(__uint_as_float(v[4 * e]) * mul, __uint_as_float(v[4 * e + 1]) * mul,
+                              __uint_as_float(v[4 * e + 2]) * mul,
+                              __uint_as_float(v[4 * e + 3]) * mul);
+          }
         }
       }
     }
@@ -580,7 +664,20 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.dq_free);
       const int pl = item_plane(i), q0 = row0 + item_q0(i);
-      if constexpr (D == 128) {
+      if constexpr (D == 128 && FA_BWD_DQ_RED) {
+        // lane = head-dim column d = 32*wq + lane; v[q] for q = 0..63: each
+        // warp instruction adds one 128-byte piece of a dQ row (32
+        // consecutive columns); rows at or past the end are skipped
+        const int dcol = 32 * wq + lane;
+        const int qlim = N - item_q0(i);
+#pragma unroll
+        for (int q = 0; q < MQ; ++q) {
+          if (q < qlim) {
+            const size_t rowi = kVarlen ? (size_t)(q0 + q) * p.Hq + pl : (size_t)pl * p.N + q0 + q;
+            atomicAdd(p.dqacc + rowi * D + dcol, __uint_as_float(v[q]) * sc);
+          }
+        }
+      } else if constexpr (D == 128) {
         // lane = head-dim column d = 32*wq + lane; v[q] for q = 0..63. Two
         // 16 KB halves: warps 0-1 stage d 0..63, then warps 2-3 stage 64..127.
         uint8_t* box = stg + (wq & 1) * C::kStgBox + (lane & 3) * 4;
@@ -653,6 +750,16 @@ cudaError_t launch(const Problem& pr) {
       !make_seq_tmap(&kp.tdq, pr, pr.dQacc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, pr.Hq, 32, C::MQ,
                      sw))
     return cudaErrorInvalidValue;
+  {
+    // dK / dV epilogue (dense batches): boxes of 128 bytes x 128 rows
+    const bool gb = pr.grad_dtype == 1;
+    const auto gt = gb ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+    const int es = gb ? 2 : 4;
+    if (!pr.cu && (!make_seq_tmap(&kp.tdk, pr, pr.dK, gt, es, pr.Hkv, 128 / es, kBN, sw) ||
+                   !make_seq_tmap(&kp.tdv, pr, pr.dV, gt, es, pr.Hkv, 128 / es, kBN, sw)))
+      return cudaErrorInvalidValue;
+  }
+  kp.dqacc = pr.dQacc;
   kp.lse2 = pr.LSE2ws;
   kp.dvec = pr.Dws;
   kp.dK = pr.dK;

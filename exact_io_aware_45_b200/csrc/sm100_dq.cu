@@ -49,6 +49,8 @@ struct Cfg {
   static constexpr int kOffK = kOffDO + kQBytes;
   static constexpr int kOffV = kOffK + kStages * kTileBytes;
   static constexpr int kOffEnd = kOffV + kStages * kTileBytes;
+  // the epilogue stages fp32 dQ (128 rows x D) over the Q and dO tiles
+  static_assert(kOffK - kOffQ >= kBM * D * 4, "epilogue staging");
 };
 
 struct alignas(16) Ctl {
@@ -69,6 +71,7 @@ constexpr uint16_t kFullBit = 0x8000;
 
 struct DqParams {
   CUtensorMap tq, tdo, tk, tv;   // [B*H][N][d] bf16, box {64, 128, 1}, 128B swizzle
+  CUtensorMap tdq;               // dQ [B*Hq][N][d] grad dtype, box {128 bytes, 128}, 128B swizzle
   const float* lse2;             // [B*Hq][Npad]
   const float* dvec;             // [B*Hq][Npad]
   void* dQ;                      // [B*Hq][N][d], fp32 or bf16
@@ -277,9 +280,13 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
       mbar_wait(&ctl.dq_done, 0, g);
       tc_fence_after();
     }
-    // tcgen05.ld is warp-collective: every lane loads, only rows < N store.
-    const bool valid = row < N;
-    const size_t orow = ((size_t)bh * N + (valid ? row : 0)) * D;
+    // scale * dQ through the shared memory of the Q and dO tiles (every MMA
+    // has completed), in the TMA's 128-byte-swizzled layout (box b of 128
+    // bytes per row at b * 16 KB, row r at r * 128, 16-byte chunk c at
+    // ((c ^ (r & 7)) << 4)), then TMA stores of whole lines; rows at or past
+    // N are clipped by the tensor map. tcgen05.ld is warp-collective: every
+    // lane loads.
+    uint8_t* st = tiles_base + C::kOffQ;
 #pragma unroll 1
     for (int cc = 0; cc < D / 32; ++cc) {
       uint32_t v[32];
@@ -289,26 +296,38 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[e] = 0u;
       }
-      if (!valid) continue;
       if (p.grad_bf16) {
         uint32_t w[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e)
           w[e] = pack_bf16(__uint_as_float(v[2 * e]) * p.scale,
                            __uint_as_float(v[2 * e + 1]) * p.scale);
-        uint4* out = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.dQ) + orow + cc * 32);
+        uint8_t* rowp = st + (cc >> 1) * 16384 + r * 128;
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-          out[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+        for (int q = 0; q < 4; ++q) {
+          const int c = 4 * (cc & 1) + q;
+          *reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4)) =
+              make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
       } else {
-        float4* out = reinterpret_cast<float4*>(static_cast<float*>(p.dQ) + orow + cc * 32);
+        uint8_t* rowp = st + cc * 16384 + r * 128;
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          out[e] = make_float4(__uint_as_float(v[4 * e]) * p.scale,
-                               __uint_as_float(v[4 * e + 1]) * p.scale,
-                               __uint_as_float(v[4 * e + 2]) * p.scale,
-                               __uint_as_float(v[4 * e + 3]) * p.scale);
+        for (int c = 0; c < 8; ++c)
+          *reinterpret_cast<float4*>(rowp + ((c ^ (r & 7)) << 4)) =
+              make_float4(__uint_as_float(v[4 * c]) * p.scale, __uint_as_float(v[4 * c + 1]) * p.scale,
+                          __uint_as_float(v[4 * c + 2]) * p.scale,
+                          __uint_as_float(v[4 * c + 3]) * p.scale);
       }
+    }
+    fence_async_smem();
+    named_sync(1, 128);
+    if (warp == 4 && lane == 0) {
+      const int esz = p.grad_bf16 ? 2 : 4;
+      const int boxes = D * esz / 128, box_cols = 128 / esz;
+      for (int bx = 0; bx < boxes; ++bx)
+        tma_store_3d(&p.tdq, st + bx * 16384, bx * box_cols, q0, bh);
+      bulk_commit();
+      bulk_wait_read0();   // the staging is read before the CTA exits
     }
   }
 
@@ -333,6 +352,13 @@ cudaError_t launch(const Problem& pr) {
       !make_tmap_3d(&kp.tk, pr.K, bf, 2, D, pr.N, BHk, 64, kBN, sw) ||
       !make_tmap_3d(&kp.tv, pr.V, bf, 2, D, pr.N, BHk, 64, kBN, sw))
     return cudaErrorInvalidValue;
+  {
+    const bool gb = pr.grad_dtype == 1;
+    const int es = gb ? 2 : 4;
+    if (!make_tmap_3d(&kp.tdq, pr.dQ, gb ? bf : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, es, D, pr.N, BHq,
+                      128 / es, kBM, sw))
+      return cudaErrorInvalidValue;
+  }
   kp.lse2 = pr.LSE2ws;
   kp.dvec = pr.Dws;
   kp.dQ = pr.dQ;

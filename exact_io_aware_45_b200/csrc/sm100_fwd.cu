@@ -81,7 +81,7 @@ constexpr int kMaxSlots = 10;     // most K/V ring slots of any form
 #endif
 // 1: dense and causal launches run the persistent form (one CTA per SM).
 #ifndef FA_FWD_PERSIST
-#define FA_FWD_PERSIST 1
+#define FA_FWD_PERSIST 0
 #endif
 
 template <int D, bool kSkip>
@@ -120,7 +120,7 @@ struct alignas(16) CtlCore {
   uint64_t q_full;
   uint64_t kv_full[kMaxSlots], kv_empty[kMaxSlots];
   uint64_t s_full[2], p_half[2], p_full[2];
-  uint64_t o_ready[2];       // query tile t's last P V has completed (skipping form)
+  uint64_t o_ready[2];       // query tile t's last P V has completed
   uint64_t o_done;
   uint64_t never;            // signalled by nothing (wait-limit test hook)
   uint64_t qt_full[2], qt_empty[2];   // per query tile Q buffer (persistent form)
@@ -152,6 +152,7 @@ struct Ctl<true> : CtlCore {
 
 struct FwdParams {
   CUtensorMap tq, tk, tv;    // [B*H][N][d] bf16, box {64, 128, 1}, 128B swizzle
+  CUtensorMap to;            // O, the same layout (dense batches: TMA-stored epilogue)
   __nv_bfloat16* O;
   float* LSE;
   const uint8_t* mask;
@@ -266,6 +267,38 @@ __device__ __forceinline__ void softmax_tile(uint32_t (&sr)[128], bool need_mask
   if (lane == 0) mbar_arrive(p_full);
 }
 
+// Writes this thread's output row O = acc / l (bf16; zeros when no P V ran
+// into the accumulator) into a 128-row tile staged in shared memory in the
+// TMA's 128-byte-swizzled layout: 64-column block cb at cb * 16 KB, row r at
+// r * 128 bytes, 16-byte chunk c of the row at ((c ^ (r & 7)) << 4). One TMA
+// store per column block then writes whole lines of O.
+template <int D>
+__device__ __forceinline__ void stage_row(uint32_t oreg, bool have_o, float l, int r,
+                                          uint8_t* stage) {
+  const float inv = (l > 0.f) ? 1.f / l : 0.f;
+#pragma unroll
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t o[32];
+    if (have_o) {
+      tmem_ld32(oreg + cc * 32, o);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) o[i] = 0u;
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i)
+      w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+    uint8_t* rowp = stage + (cc >> 1) * 16384 + r * 128;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int c = 4 * (cc & 1) + q;
+      *reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4)) =
+          make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+    }
+  }
+}
+
 // Stores this thread's output row: O = acc / l (bf16, 16-byte vectors) from
 // the TMEM accumulator (or zeros when no P V ran into it) and LSE =
 // (m_ref + log2 l) ln 2 (-inf for a row with no visible key).
@@ -318,14 +351,6 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   // inside a chunk the query blocks with the longest causal rows start first.
   int bh, rblk;
   chunked_order(blockIdx.x, p.nblk, p.BH, p.chunk, bh, rblk);
-  // A launch whose error word is already set (an earlier wait ran out and
-  // nobody has read the word yet) does no work: its inputs may be invalid.
-  // One thread reads the word and the whole CTA leaves together, before any
-  // barrier is initialised or TMEM allocated (another CTA may set the word
-  // meanwhile, so per-thread reads could disagree).
-  if (threadIdx.x == 0) ctl.skip = (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) ? 1 : 0;
-  __syncthreads();
-  if (ctl.skip) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int blk = p.nblk - 1 - rblk;
   const int h = bh % p.Hq, b = bh / p.Hq;
@@ -352,7 +377,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   // 0 .. kb_end-1 and needs no storage.
   const int kb_end = min(nb, mod_last_key(p.mod, qb1 * kBM + kBM - 1, N) / kBN + 1);
 
+  // K/V ring loads issued before the block barrier below (lockstep form)
+  const int pre_loads = kSkip ? 0 : min(kSlots, 2 * kb_end);
   if (threadIdx.x == 0) {
+    // A launch whose error word is already set (an earlier wait ran out and
+    // nobody has read the word yet) does no work: its inputs may be invalid.
+    // This one thread reads the word (while it sets up the barriers) and the
+    // whole CTA leaves together after the block barrier below, before any
+    // wait (another CTA may set the word meanwhile, so per-thread reads
+    // could disagree).
+    const unsigned err_word = *reinterpret_cast<volatile unsigned*>(p.err);
     mbar_init(&ctl.q_full, 1);
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&ctl.kv_full[s], 1);
@@ -369,6 +403,27 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     ctl.abort = 0;
     if constexpr (!kSkip) ctl.ntiles = kb_end;
     fence_mbar_init();
+    ctl.skip = err_word != 0u;
+    if (!ctl.skip) {
+      // This thread is also the TMA producer: the Q tiles and, in the
+      // lockstep form, the first K/V ring loads start now, so their latency
+      // overlaps the TMEM allocation, the tile lists and the block barrier.
+      prefetch_tmap(&p.tq);
+      prefetch_tmap(&p.tk);
+      prefetch_tmap(&p.tv);
+      mbar_expect_tx(&ctl.q_full, 2 * C::kQBytes);
+      for (int t = 0; t < 2; ++t)
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_load_3d(tiles_base + C::kOffQ + t * C::kQBytes + cb * C::kBlockBytes, &p.tq,
+                      &ctl.q_full, cb * 64, row0 + q0 + t * kBM, qplane);
+      for (int n = 0; n < pre_loads; ++n) {
+        mbar_expect_tx(&ctl.kv_full[n], C::kTileBytes);
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_load_3d(tiles_base + C::kOffKV + n * C::kTileBytes + cb * C::kBlockBytes,
+                      (n & 1) ? &p.tv : &p.tk, &ctl.kv_full[n], cb * 64, row0 + (n >> 1) * kBN,
+                      kplane);
+      }
+    }
   }
   if (warp == 2) {
     tmem_alloc(&ctl.tmem_base, 512);
@@ -421,6 +476,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = ctl.tmem_base;
+  if (ctl.skip) {   // the error word was set at launch: nothing was issued
+    if (warp == 2) tmem_dealloc(tm, 512);
+    return;
+  }
   const int T = ctl.ntiles;
   const Guard g{&ctl.abort, p.err};
   // j-th key tile of the CTA's list
@@ -431,19 +490,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0 && T > 0) {
-      prefetch_tmap(&p.tq);
-      prefetch_tmap(&p.tk);
-      prefetch_tmap(&p.tv);
-      mbar_expect_tx(&ctl.q_full, 2 * C::kQBytes);
-      for (int t = 0; t < 2; ++t)
-        for (int cb = 0; cb < C::kColBlocks; ++cb)
-          tma_load_3d(tiles_base + C::kOffQ + t * C::kQBytes + cb * C::kBlockBytes, &p.tq,
-                      &ctl.q_full, cb * 64, row0 + q0 + t * kBM, qplane);
-      // K_0, V_0, K_1, V_1, ... into the slot ring, each slot reused once the
-      // MMA warp has released the tile kSlots loads earlier.
-      int issued = 0;
-      for (int n = 0; n < 2 * T; ++n) {
+    if (lane == 0) {
+      // (Q and the first pre_loads ring tiles were issued before the block
+      // barrier.) K_0, V_0, K_1, V_1, ... into the slot ring, each slot
+      // reused once the MMA warp has released the tile kSlots loads earlier.
+      int issued = pre_loads;
+      for (int n = pre_loads; n < 2 * T; ++n) {
         const int s = ring_slot<kSlots>(n);
         if (n >= kSlots && !mbar_wait(&ctl.kv_empty[s], ring_phase<kSlots>(n - kSlots), g)) break;
         const int kb = tile_of(n >> 1);
@@ -580,6 +632,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           tc_fence_after();
           issue_pv(0, j, j > 0, 1);
           const bool more = j + 1 < T;
+          // the last P V of a query tile: its epilogue may start
+          if (!more) mma_commit(&ctl.o_ready[0]);
           if (more) {
             if (!(ok = wait_tile(2 * j + 2))) break;
             tc_fence_after();
@@ -592,6 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           if (!(ok = mbar_wait(&ctl.p_full[1], j & 1, g))) break;
           tc_fence_after();
           issue_pv(1, j, j > 0, 1);
+          if (!more) mma_commit(&ctl.o_ready[1]);
           release_tile(2 * j + 1);   // V_j
           if (more) {
             issue_s(1, j + 1);
@@ -676,16 +731,41 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     else
       have_o = T > 0;
     if (have_o) {
-      mbar_wait(kSkip ? &ctl.o_ready[t] : &ctl.o_done, 0, g);
+      // this query tile's last P V has completed (its S MMAs, which read the
+      // Q buffer, came before it)
+      mbar_wait(&ctl.o_ready[t], 0, g);
       tc_fence_after();
+    } else {
+      // no MMA read this tile's Q buffer, but its load may still be landing:
+      // wait for it before the buffer is reused for the output
+      mbar_wait(&ctl.q_full, 0, g);
     }
     const bool valid = row < N;
-    // O rows: [B][H][N][d] (dense) or [total][H][d] (variable-length)
-    const size_t o_base = kVarlen ? ((size_t)row0 * p.Hq + h) * D : (size_t)bh * p.N * D;
-    const size_t o_rs = kVarlen ? (size_t)p.Hq * D : (size_t)D;
-    const size_t lse_base = kVarlen ? (size_t)h * p.total + row0 : (size_t)bh * p.N;
-    store_row<D>(oreg, have_o, m_ref, l, valid, p.O + o_base + (size_t)(valid ? row : 0) * o_rs,
-                 p.LSE + lse_base + (valid ? row : 0));
+    if constexpr (!kVarlen) {
+      // O through the free Q buffer of this tile and TMA stores (rows at or
+      // past N are clipped by the tensor map); LSE row by row
+      uint8_t* stage = tiles_base + C::kOffQ + t * C::kQBytes;
+      stage_row<D>(oreg, have_o, l, r, stage);
+      if (valid)
+        p.LSE[(size_t)bh * p.N + row] = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+      fence_async_smem();
+      named_sync(1 + t, 128);
+      if (warp == 4 + 4 * t && lane == 0) {
+#pragma unroll
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_store_3d(&p.to, stage + cb * C::kBlockBytes, cb * 64, tile_row0, bh);
+        bulk_commit();
+        bulk_wait_read0();   // the staging buffer is read before the CTA exits
+      }
+    } else {
+      // packed batch: a 128-row box could reach into the next sequence, so
+      // rows are stored one by one ([total][H][d])
+      const size_t o_base = ((size_t)row0 * p.Hq + h) * D;
+      const size_t lse_base = (size_t)h * p.total + row0;
+      store_row<D>(oreg, have_o, m_ref, l, valid,
+                   p.O + o_base + (size_t)(valid ? row : 0) * p.Hq * D,
+                   p.LSE + lse_base + (valid ? row : 0));
+    }
   }
 
   tc_fence_before();
@@ -907,12 +987,16 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
     bool ok = true;
     int nt = 0, k = 0;
     for (int w = blockIdx.x; ok && w < W; w += gridDim.x, ++k) {
-      const Item it = item_of(w);
-      const int tile_row0 = it.q0 + t * kBM;
+      int tile_row0, T;
+      {
+        const Item it = item_of(w);
+        tile_row0 = it.q0 + t * kBM;
+        T = it.T;
+      }
       const int row = tile_row0 + r;
       const bool tile_live = tile_row0 < N;   // the second tile may lie past the end
       float m_ref = -INFINITY, l = 0.f;
-      for (int j = 0; j < it.T; ++j) {
+      for (int j = 0; j < T; ++j) {
         if (!(ok = mbar_wait(&ctl.s_full[t], (nt + j) & 1, g))) break;
         tc_fence_after();
         uint32_t sr[128];
@@ -942,14 +1026,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
                                       &ctl.p_half[t], &ctl.p_full[t], lane);
       }
       if (!ok) break;
-      nt += it.T;
+      nt += T;
       // epilogue of this item: the last P V of this query tile has completed
       if (!(ok = mbar_wait(&ctl.o_ready[t], k & 1, g))) break;
       tc_fence_after();
       const bool valid = row < N;
-      store_row<D>(oreg, true, m_ref, l, valid,
-                   p.O + ((size_t)it.bh * N + (valid ? row : 0)) * D,
-                   p.LSE + (size_t)it.bh * N + (valid ? row : 0));
+      const size_t bh = (size_t)item_of(w).bh;
+      store_row<D>(oreg, true, m_ref, l, valid, p.O + (bh * N + (valid ? row : 0)) * D,
+                   p.LSE + bh * N + (valid ? row : 0));
     }
   }
 
@@ -979,7 +1063,8 @@ cudaError_t launch(const Problem& pr) {
   const auto sw = CU_TENSOR_MAP_SWIZZLE_128B;
   if (!make_seq_tmap(&kp.tq, pr, pr.Q, bf, 2, pr.Hq, 64, kBM, sw) ||
       !make_seq_tmap(&kp.tk, pr, pr.K, bf, 2, pr.Hkv, 64, kBN, sw) ||
-      !make_seq_tmap(&kp.tv, pr, pr.V, bf, 2, pr.Hkv, 64, kBN, sw))
+      !make_seq_tmap(&kp.tv, pr, pr.V, bf, 2, pr.Hkv, 64, kBN, sw) ||
+      !make_seq_tmap(&kp.to, pr, pr.Oout, bf, 2, pr.Hq, 64, kBM, sw))
     return cudaErrorInvalidValue;
   kp.O = static_cast<__nv_bfloat16*>(pr.Oout);
   kp.LSE = pr.LSEout;
