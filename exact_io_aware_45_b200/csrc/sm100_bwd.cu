@@ -61,11 +61,10 @@ constexpr int kChunk = FA_BWD_CHUNK;
 #ifndef FA_BWD_ITEM_SPLIT
 #define FA_BWD_ITEM_SPLIT 0
 #endif
-// 1: at d = 128 the dQ drain adds into the fp32 accumulator with red.global
-// from registers instead of staging in shared memory for TMA reduce-adds
-// (build-time choice for A/B measurements).
-#ifndef FA_BWD_DQ_RED
-#define FA_BWD_DQ_RED 0
+// d = 128, dense batches: 1 lets the dQ drain warps stage and store dV while
+// the softmax warps do dK (0: the softmax warps do both, one after the other).
+#ifndef FA_BWD_DV_DRAIN
+#define FA_BWD_DV_DRAIN 1
 #endif
 constexpr float kLog2e = 1.4426950408889634f;
 
@@ -82,6 +81,7 @@ struct Cfg {
   static constexpr int kSoftWarps = (D == 64 || kItemSplit) ? 8 : 4;
   static constexpr int kColHalves = (D == 64) ? 2 : 1;    // groups sharing an item's columns
   static constexpr int kThreads = (8 + kSoftWarps) * 32;
+  static constexpr bool kDrainDV = kSoftWarps == 4 && FA_BWD_DV_DRAIN;
   static constexpr bool kDbl = (D == 128);                // two S/dP sets in TMEM
   static constexpr int MQ = (D == 64) ? 128 : 64;         // query rows per item
   static constexpr int kStages = kDbl ? 3 : 2;            // Q / dO ring depth
@@ -128,6 +128,48 @@ struct alignas(16) Ctl {
 // visible, so its scores need no masking.
 constexpr uint16_t kFullBit = 0x8000;
 
+// Stages one thread's row r of a 128 x D gradient accumulator (TMEM columns
+// from taddr; zeros when the CTA ran no item) at st, in the TMA's
+// 128-byte-swizzled layout: box b (128 bytes of each row: 32 fp32 or 64 bf16
+// columns) at b * 16 KB, row r at r * 128 bytes, 16-byte chunk c at
+// ((c ^ (r & 7)) << 4).
+template <int D>
+__device__ __forceinline__ void stage_grad(uint8_t* st, uint32_t taddr, bool have, float mul,
+                                           bool grad_bf16, int r) {
+#pragma unroll 1
+  for (int cc = 0; cc < D / 32; ++cc) {
+    uint32_t v[32];
+    if (have) {
+      tmem_ld32(taddr + cc * 32, v);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] = 0u;
+    }
+    if (grad_bf16) {
+      // 32 columns = 64 bytes: chunks 4 (cc & 1) .. +3 of box cc / 2
+      uint32_t w[16];
+#pragma unroll
+      for (int e = 0; e < 16; ++e)
+        w[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
+      uint8_t* rowp = st + (cc >> 1) * 16384 + r * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c = 4 * (cc & 1) + q;
+        *reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4)) =
+            make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      }
+    } else {
+      // 32 columns = 128 bytes: all 8 chunks of box cc
+      uint8_t* rowp = st + cc * 16384 + r * 128;
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<float4*>(rowp + ((c ^ (r & 7)) << 4)) =
+            make_float4(__uint_as_float(v[4 * c]) * mul, __uint_as_float(v[4 * c + 1]) * mul,
+                        __uint_as_float(v[4 * c + 2]) * mul, __uint_as_float(v[4 * c + 3]) * mul);
+    }
+  }
+}
+
 struct BwdParams {
   CUtensorMap tq, tdo;         // [B*Hq][N][d] bf16, box {64, MQ}, 128B swizzle
   CUtensorMap tk, tv;          // [B*Hkv][N][d] bf16, box {64, 128}
@@ -135,7 +177,6 @@ struct BwdParams {
   CUtensorMap tdk, tdv;        // [B*Hkv][N][d] grad dtype, box {128 bytes, 128}, 128B swizzle
   const float* lse2;           // [B*Hq][Npad]
   const float* dvec;           // [B*Hq][Npad]
-  float* dqacc;                // the fp32 dQ accumulator (layout of tdq)
   void* dK;
   void* dV;
   const uint8_t* mask;
@@ -213,11 +254,11 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
     mbar_init(&ctl.never, 1);
     ctl.abort = 0;
     fence_mbar_init();
-    ctl.skip = err_word != 0u;
-    if (!ctl.skip) {
+    {
       // This thread is also the TMA producer: the K and V tiles start now, so
-      // their latency overlaps the TMEM allocation, the query-tile list and
-      // the block barrier.
+      // their latency (and that of the error-word read) overlaps the TMEM
+      // allocation, the query-tile list and the block barrier. A CTA that
+      // then finds the word set waits for them to land and does nothing else.
       prefetch_tmap(&p.tk);
       prefetch_tmap(&p.tv);
       mbar_expect_tx(&ctl.kv_full, 2 * C::kKVBytes);
@@ -228,6 +269,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
                     kplane);
       }
     }
+    ctl.skip = err_word != 0u;
   }
   if (warp == 2) {
     tmem_alloc(&ctl.tmem_base, 512);
@@ -258,7 +300,8 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = ctl.tmem_base;
-  if (ctl.skip) {   // the error word was set at launch: nothing was issued
+  if (ctl.skip) {   // the error word was set at launch: no work
+    if (threadIdx.x == 0) drain_wait(&ctl.kv_full, 0);
     if (warp == 2) tmem_dealloc(tm, 512);
     return;
   }
@@ -543,62 +586,27 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       tc_fence_after();
     }
     const bool valid = kv < N;
-    // 8 softmax warps: warps 4-7 store dK, warps 8-11 dV; 4: warps 4-7 both.
+    // 8 softmax warps: warps 4-7 store dK, warps 8-11 dV. 4 (d = 128): warps
+    // 4-7 store dK and the dQ drain warps dV (both for packed batches).
     const int which_lo = (C::kSoftWarps == 8) ? half : 0;
-    const int which_hi = (C::kSoftWarps == 8) ? half + 1 : 2;
+    const int which_hi = (C::kSoftWarps == 8) ? half + 1 : (!kVarlen && C::kDrainDV ? 1 : 2);
     if constexpr (!kVarlen) {
-      // dK and dV through the shared memory of the Q/dO ring and the dS
-      // buffers (every MMA has completed), in the TMA's 128-byte-swizzled
-      // layout: box b (128 bytes of each row: 32 fp32 or 64 bf16 columns) at
-      // b * 16 KB, row r at r * 128 bytes, 16-byte chunk c at ((c ^ (r & 7))
-      // << 4); dK first, dV after it. One thread then stores whole lines with
-      // TMA (rows at or past N are clipped by the tensor map).
+      // dK (and dV) through the shared memory of the Q/dO ring and the dS
+      // buffers (every MMA has completed): dK at the start, dV one staged
+      // tensor after it. Each warpgroup's first thread then stores its
+      // tensor's whole lines with TMA (rows at or past N are clipped by the
+      // tensor map).
       const int esz = p.grad_bf16 ? 2 : 4;
       const int tbytes = kBN * D * esz;   // one staged tensor
 #pragma unroll 1
-      for (int which = which_lo; which < which_hi; ++which) {
-        const uint32_t col = which ? C::kDV : C::kDK;
-        const float mul = which ? 1.f : p.scale;
-        uint8_t* st = base + C::kOffQ + which * tbytes;
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t v[32];
-          if (n_items > 0) {
-            tmem_ld32(tm + col + lane_off + cc * 32, v);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = 0u;
-          }
-          if (p.grad_bf16) {
-            // 32 columns = 64 bytes: chunks 4 (cc & 1) .. +3 of box cc / 2
-            uint32_t w[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e)
-              w[e] = pack_bf16(__uint_as_float(v[2 * e]) * mul, __uint_as_float(v[2 * e + 1]) * mul);
-            uint8_t* rowp = st + (cc >> 1) * 16384 + r * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int c = 4 * (cc & 1) + q;
-              *reinterpret_cast<uint4*>(rowp + ((c ^ (r & 7)) << 4)) =
-                  make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-            }
-          } else {
-            // 32 columns = 128 bytes: all 8 chunks of box cc
-            uint8_t* rowp = st + cc * 16384 + r * 128;
-#pragma unroll
-            for (int c = 0; c < 8; ++c)
-              *reinterpret_cast<float4*>(rowp + ((c ^ (r & 7)) << 4)) =
-                  make_float4(__uint_as_float(v[4 * c]) * mul, __uint_as_float(v[4 * c + 1]) * mul,
-                              __uint_as_float(v[4 * c + 2]) * mul,
-                              __uint_as_float(v[4 * c + 3]) * mul);
-          }
-        }
-      }
+      for (int which = which_lo; which < which_hi; ++which)
+        stage_grad<D>(base + C::kOffQ + which * tbytes, tm + (which ? C::kDV : C::kDK) + lane_off,
+                      n_items > 0, which ? 1.f : p.scale, p.grad_bf16, r);
       fence_async_smem();
-      named_sync(2, C::kSoftWarps * 32);
-      if (warp == 4 && lane == 0) {
+      named_sync(2 + half, 128);
+      if (wq == 0 && lane == 0) {
         const int boxes = D * esz / 128, box_cols = 128 / esz;
-        for (int which = 0; which < 2; ++which)
+        for (int which = which_lo; which < which_hi; ++which)
           for (int bx = 0; bx < boxes; ++bx)
             tma_store_3d(which ? &p.tdv : &p.tdk, base + C::kOffQ + which * tbytes + bx * 16384,
                          bx * box_cols, n0, bhk);
@@ -664,20 +672,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.dq_free);
       const int pl = item_plane(i), q0 = row0 + item_q0(i);
-      if constexpr (D == 128 && FA_BWD_DQ_RED) {
-        // lane = head-dim column d = 32*wq + lane; v[q] for q = 0..63: each
-        // warp instruction adds one 128-byte piece of a dQ row (32
-        // consecutive columns); rows at or past the end are skipped
-        const int dcol = 32 * wq + lane;
-        const int qlim = N - item_q0(i);
-#pragma unroll
-        for (int q = 0; q < MQ; ++q) {
-          if (q < qlim) {
-            const size_t rowi = kVarlen ? (size_t)(q0 + q) * p.Hq + pl : (size_t)pl * p.N + q0 + q;
-            atomicAdd(p.dqacc + rowi * D + dcol, __uint_as_float(v[q]) * sc);
-          }
-        }
-      } else if constexpr (D == 128) {
+      if constexpr (D == 128) {
         // lane = head-dim column d = 32*wq + lane; v[q] for q = 0..63. Two
         // 16 KB halves: warps 0-1 stage d 0..63, then warps 2-3 stage 64..127.
         uint8_t* box = stg + (wq & 1) * C::kStgBox + (lane & 3) * 4;
@@ -724,6 +719,26 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
         }
       }
     }
+    if constexpr (!kVarlen && C::kDrainDV) {
+      // dV epilogue, beside the softmax warps' dK: staged one tensor after
+      // dK, clear of the dQ staging
+      if (n_items > 0) {
+        mbar_wait(&ctl.acc_done, 0, g);
+        tc_fence_after();
+      }
+      const int esz = p.grad_bf16 ? 2 : 4;
+      const int tbytes = kBN * D * esz;
+      stage_grad<D>(base + C::kOffQ + tbytes, tm + C::kDV + lane_off, n_items > 0, 1.f,
+                    p.grad_bf16, wq * 32 + lane);
+      fence_async_smem();
+      named_sync(1, 128);
+      if (leader) {
+        const int boxes = D * esz / 128, box_cols = 128 / esz;
+        for (int bx = 0; bx < boxes; ++bx)
+          tma_store_3d(&p.tdv, base + C::kOffQ + tbytes + bx * 16384, bx * box_cols, n0, bhk);
+        bulk_commit();
+      }
+    }
     if (leader) bulk_wait0();
   }
 
@@ -759,7 +774,6 @@ cudaError_t launch(const Problem& pr) {
                    !make_seq_tmap(&kp.tdv, pr, pr.dV, gt, es, pr.Hkv, 128 / es, kBN, sw)))
       return cudaErrorInvalidValue;
   }
-  kp.dqacc = pr.dQacc;
   kp.lse2 = pr.LSE2ws;
   kp.dvec = pr.Dws;
   kp.dK = pr.dK;

@@ -79,9 +79,13 @@ constexpr int kMaxSlots = 10;     // most K/V ring slots of any form
 #ifndef FA_FWD_EMU_PAIRS_D128
 #define FA_FWD_EMU_PAIRS_D128 0
 #endif
-// 1: dense and causal launches run the persistent form (one CTA per SM).
-#ifndef FA_FWD_PERSIST
-#define FA_FWD_PERSIST 0
+// Dense and causal launches with N up to this many keys run the persistent
+// form (one CTA per SM over a queue of items), the others one CTA per item:
+// measured on B200, the persistent form is 1-13% faster up to N = 4096 (the
+// fixed cost per item matters most there) and 3-6% slower at 8K-16K (its
+// steady state is a little slower). 0: never persistent.
+#ifndef FA_FWD_PERSIST_MAXN
+#define FA_FWD_PERSIST_MAXN 4096
 #endif
 
 template <int D, bool kSkip>
@@ -124,6 +128,8 @@ struct alignas(16) CtlCore {
   uint64_t o_done;
   uint64_t never;            // signalled by nothing (wait-limit test hook)
   uint64_t qt_full[2], qt_empty[2];   // per query tile Q buffer (persistent form)
+  uint64_t item_full[4], item_empty[4];   // work-item ring (persistent form)
+  int item_id[4];
   uint32_t tmem_base;
   int abort;
   int skip;                  // the error word was set at launch: the CTA does nothing
@@ -377,8 +383,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   // 0 .. kb_end-1 and needs no storage.
   const int kb_end = min(nb, mod_last_key(p.mod, qb1 * kBM + kBM - 1, N) / kBN + 1);
 
-  // K/V ring loads issued before the block barrier below (lockstep form)
-  const int pre_loads = kSkip ? 0 : min(kSlots, 2 * kb_end);
+  // K/V ring loads issued before the block barrier below (lockstep form):
+  // K_0 only, so the other threads do not wait long at the barrier for the
+  // issuing thread
+  const int pre_loads = kSkip ? 0 : 1;
   if (threadIdx.x == 0) {
     // A launch whose error word is already set (an earlier wait ran out and
     // nobody has read the word yet) does no work: its inputs may be invalid.
@@ -403,11 +411,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     ctl.abort = 0;
     if constexpr (!kSkip) ctl.ntiles = kb_end;
     fence_mbar_init();
-    ctl.skip = err_word != 0u;
-    if (!ctl.skip) {
+    {
       // This thread is also the TMA producer: the Q tiles and, in the
-      // lockstep form, the first K/V ring loads start now, so their latency
-      // overlaps the TMEM allocation, the tile lists and the block barrier.
+      // lockstep form, K_0 start now, so their latency (and that of the
+      // error-word read) overlaps the TMEM allocation, the tile lists and the
+      // block barrier. A CTA that then finds the word set waits for these
+      // copies to land and does nothing else.
       prefetch_tmap(&p.tq);
       prefetch_tmap(&p.tk);
       prefetch_tmap(&p.tv);
@@ -424,6 +433,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
                       kplane);
       }
     }
+    ctl.skip = err_word != 0u;
   }
   if (warp == 2) {
     tmem_alloc(&ctl.tmem_base, 512);
@@ -476,7 +486,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = ctl.tmem_base;
-  if (ctl.skip) {   // the error word was set at launch: nothing was issued
+  if (ctl.skip) {   // the error word was set at launch: no work
+    if (threadIdx.x == 0) {
+      drain_wait(&ctl.q_full, 0);
+      for (int n = 0; n < pre_loads; ++n) drain_wait(&ctl.kv_full[n], 0);
+    }
     if (warp == 2) tmem_dealloc(tm, 512);
     return;
   }
@@ -776,34 +790,57 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
   }
 }
 
-// Persistent form of the lockstep forward (dense and causal launches, no
-// mask, window left edge or documents): one CTA per SM walks a static list
-// of work items (a (batch, head) and a block of two 128-row query tiles, in
-// the launch order of the one-item form: groups of heads that share L2,
-// longest causal blocks first), item w = blockIdx.x + k * gridDim.x. What a
-// CTA of the one-item form pays once per item is overlapped here with the
-// previous item: the Q tile t of item k+1 is loaded as soon as the last S_t
-// of item k has read the old one (qt_empty[t]), the K/V slot ring runs on
-// across items, the next item's first S is issued right after the last P V
-// of the current one, and the epilogue of item k (O from TMEM to global
-// memory) runs while the MMA warp works on item k+1. Barrier phases count
-// tiles and items per CTA; the per-item softmax state starts afresh.
+// Persistent form of the lockstep forward (dense and causal launches without
+// a block mask, left window edge or documents): one CTA per SM takes work
+// items (a (batch, head) and a block of two 128-row query tiles, numbered in
+// the launch order of the one-item form) from a queue, so what a CTA of the
+// one-item form pays per item -- set-up, the first S waiting for Q, the
+// epilogue with the tensor core idle, the gap before the next CTA starts --
+// is paid once per SM or overlapped:
+//  * the producer draws item numbers from a counter in the workspace's
+//    error block (atomicAdd), which balances causal items of different
+//    lengths, and hands them to the MMA and softmax warps through a ring of
+//    kItemRing entries; the last CTA to leave resets the counter;
+//  * the Q tile t of the next item is loaded as soon as the last S_t of the
+//    current one has read the buffer, and the K/V ring runs on across items;
+//  * the epilogue stages O in a buffer of its own and writes it with TMA
+//    stores, so the next item's Q is not disturbed.
+// Barrier phases count tiles and items per CTA; each item's softmax state
+// starts afresh.
+constexpr int kItemRing = 4;
+
+template <int D>
+struct PCfg {
+  static constexpr int kSlots = (D == 64) ? 8 : 3;   // K/V ring (3 measured as fast as 5)
+  static constexpr int kTileBytes = kBN * D * 2;
+  static constexpr int kQBytes = kBM * D * 2;
+  static constexpr int kColBlocks = D / 64;
+  static constexpr int kBlockBytes = 128 * 128;
+  static constexpr int kEmuPairs = Cfg<D, false>::kEmuPairs;
+  static constexpr uint32_t kS0 = 0, kS1 = 128;
+  static constexpr uint32_t kO0 = 256, kO1 = 256 + (D == 64 ? 64 : 128);
+  static constexpr uint32_t kPOff = 64;
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffKV = 2 * kQBytes;
+  static constexpr int kOffStage = kOffKV + kSlots * kTileBytes;   // O staging, two tiles
+  static constexpr int kOffEnd = kOffStage + 2 * kQBytes;
+  static_assert(kSlots <= kMaxSlots, "ring barriers");
+};
+
 template <int D, bool kCap>
 __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_constant__ FwdParams p) {
-  using C = Cfg<D, false>;
+  using C = PCfg<D>;
   constexpr int kSlots = C::kSlots;
   extern __shared__ uint8_t smem_raw[];
   Ctl<false>& ctl = *reinterpret_cast<Ctl<false>*>(smem_raw);
   const uint32_t raw_addr = smem_u32(smem_raw);
   const uint32_t tile_addr = (raw_addr + sizeof(Ctl<false>) + 1023u) & ~1023u;
   uint8_t* tiles_base = smem_raw + (tile_addr - raw_addr);
-  // A launch whose error word is already set does no work (see fwd_kernel).
-  if (threadIdx.x == 0) ctl.skip = (*reinterpret_cast<volatile unsigned*>(p.err) != 0u) ? 1 : 0;
-  __syncthreads();
-  if (ctl.skip) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int W = p.BH * p.nblk;   // work items
   const int N = p.N, nb = p.nb;
+  unsigned* const next_item = p.err + 16;   // queue counter (workspace byte 64)
+  unsigned* const ctas_done = p.err + 17;   // CTAs that have left (byte 68)
 
   // item w -> (bh, first query row, number of key tiles, kv plane)
   struct Item {
@@ -822,6 +859,8 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
   };
 
   if (threadIdx.x == 0) {
+    // a launch whose error word is already set does no work (see fwd_kernel)
+    const unsigned err_word = *reinterpret_cast<volatile unsigned*>(p.err);
     for (int s = 0; s < kSlots; ++s) {
       mbar_init(&ctl.kv_full[s], 1);
       mbar_init(&ctl.kv_empty[s], 1);
@@ -834,10 +873,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
       mbar_init(&ctl.p_full[t], 4);
       mbar_init(&ctl.o_ready[t], 1);
     }
+    for (int i = 0; i < kItemRing; ++i) {
+      mbar_init(&ctl.item_full[i], 1);
+      mbar_init(&ctl.item_empty[i], 9);   // the MMA thread and the eight softmax warps
+    }
     mbar_init(&ctl.o_done, 1);
     mbar_init(&ctl.never, 1);
     ctl.abort = 0;
     fence_mbar_init();
+    ctl.skip = err_word != 0u;
   }
   if (warp == 2) {
     tmem_alloc(&ctl.tmem_base, 512);
@@ -849,19 +893,31 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
   const uint32_t tm = ctl.tmem_base;
   const Guard g{&ctl.abort, p.err};
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+  if (ctl.skip) {
+    // no work
+  } else if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer + queue
     if (lane == 0) {
       prefetch_tmap(&p.tq);
       prefetch_tmap(&p.tk);
       prefetch_tmap(&p.tv);
+      prefetch_tmap(&p.to);
       int n = 0;              // K/V tiles loaded into the ring so far
       int qi[2] = {0, 0};     // loads of each Q tile buffer so far
       bool ok = true;
-      for (int w = blockIdx.x; ok && w < W; w += gridDim.x) {
-        const Item it = item_of(w);
-        // Q tile t of this item once the previous item's last S_t has read
-        // the buffer
+      for (int k = 0; ok; ++k) {
+        // the next item for this CTA (or -1: the queue is empty)
+        const int slot = k % kItemRing;
+        if (k >= kItemRing &&
+            !(ok = mbar_wait(&ctl.item_empty[slot], ((k / kItemRing) - 1) & 1, g)))
+          break;
+        const unsigned w = atomicAdd(next_item, 1u);
+        const int wi = (w < (unsigned)W) ? (int)w : -1;
+        ctl.item_id[slot] = wi;
+        mbar_arrive(&ctl.item_full[slot]);
+        if (wi < 0) break;
+        const Item it = item_of(wi);
+        // Q tile t once the previous item's last S_t has read the buffer
         for (int t = 0; ok && t < 2; ++t) {
           if (qi[t] > 0 && !(ok = mbar_wait(&ctl.qt_empty[t], (qi[t] - 1) & 1, g))) break;
           mbar_expect_tx(&ctl.qt_full[t], C::kQBytes);
@@ -874,11 +930,11 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
           const int s = ring_slot<kSlots>(n);
           if (n >= kSlots && !(ok = mbar_wait(&ctl.kv_empty[s], ring_phase<kSlots>(n - kSlots), g)))
             break;
-          const CUtensorMap* m = (j & 1) ? &p.tv : &p.tk;
           mbar_expect_tx(&ctl.kv_full[s], C::kTileBytes);
           for (int cb = 0; cb < C::kColBlocks; ++cb)
-            tma_load_3d(tiles_base + C::kOffKV + s * C::kTileBytes + cb * C::kBlockBytes, m,
-                        &ctl.kv_full[s], cb * 64, (j >> 1) * kBN, it.kplane);
+            tma_load_3d(tiles_base + C::kOffKV + s * C::kTileBytes + cb * C::kBlockBytes,
+                        (j & 1) ? &p.tv : &p.tk, &ctl.kv_full[s], cb * 64, (j >> 1) * kBN,
+                        it.kplane);
         }
       }
       // Every issued copy has landed before the CTA may exit.
@@ -923,10 +979,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
         }
       };
       bool ok = injected_stall(&ctl.never, p.stall, g);
-      int n = 0, nt = 0, k = 0;   // ring tiles, softmax tiles, items so far
-      for (int w = blockIdx.x; ok && w < W; w += gridDim.x, ++k) {
-        const Item it = item_of(w);
-        const int T = it.T;
+      int n = 0, nt = 0;   // ring tiles and softmax tiles so far
+      for (int k = 0; ok; ++k) {
+        const int slot = k % kItemRing;
+        if (!(ok = mbar_wait(&ctl.item_full[slot], (k / kItemRing) & 1, g))) break;
+        const int wi = ctl.item_id[slot];
+        mbar_arrive(&ctl.item_empty[slot]);
+        if (wi < 0) break;
+        const int T = item_of(wi).T;
         // K_j is ring tile n + 2j, V_j is n + 2j + 1
         for (int t = 0; t < 2; ++t) {
           if (!(ok = mbar_wait(&ctl.qt_full[t], k & 1, g) && wait_tile(n))) break;
@@ -985,16 +1045,22 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
     const uint32_t oreg = tm + (t ? C::kO1 : C::kO0) + lane_off;
     const float c = kCap ? 1.f : p.c;
     bool ok = true;
-    int nt = 0, k = 0;
-    for (int w = blockIdx.x; ok && w < W; w += gridDim.x, ++k) {
+    int nt = 0;
+    for (int k = 0; ok; ++k) {
+      const int slot = k % kItemRing;
+      if (!(ok = mbar_wait(&ctl.item_full[slot], (k / kItemRing) & 1, g))) break;
+      const int wi = ctl.item_id[slot];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&ctl.item_empty[slot]);
+      if (wi < 0) break;
+      // (only what the tile loop needs stays live across it; the epilogue
+      // decodes the item again)
       int tile_row0, T;
       {
-        const Item it = item_of(w);
+        const Item it = item_of(wi);
         tile_row0 = it.q0 + t * kBM;
         T = it.T;
       }
-      const int row = tile_row0 + r;
-      const bool tile_live = tile_row0 < N;   // the second tile may lie past the end
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < T; ++j) {
         if (!(ok = mbar_wait(&ctl.s_full[t], (nt + j) & 1, g))) break;
@@ -1008,14 +1074,15 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
         }
         const int col0 = j * kBN;
         // as in the lockstep form: this query tile may see none of key tile j
+        // (the second tile may also lie past the end of the sequence)
         const int wr = p.mod.wr, pre1 = p.mod.prefix - 1;
         const bool dead =
-            !tile_live || (wr >= 0 && col0 > max(tile_row0 + kBM - 1 + wr, pre1));
+            tile_row0 >= N || (wr >= 0 && col0 > max(tile_row0 + kBM - 1 + wr, pre1));
         const bool need_mask =
             dead || col0 + kBN > N || (wr >= 0 && col0 + kBN - 1 > max(tile_row0 + wr, pre1));
         if (need_mask) {
           int row_lo, row_hi;
-          mod_row_keys(p.mod, row, N, row_lo, row_hi);
+          mod_row_keys(p.mod, tile_row0 + r, N, row_lo, row_hi);
           const int lo = row_lo - col0;
           const int hi = dead ? lo - 1 : row_hi - col0;
 #pragma unroll
@@ -1030,11 +1097,23 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
       // epilogue of this item: the last P V of this query tile has completed
       if (!(ok = mbar_wait(&ctl.o_ready[t], k & 1, g))) break;
       tc_fence_after();
-      const bool valid = row < N;
-      const size_t bh = (size_t)item_of(w).bh;
-      store_row<D>(oreg, true, m_ref, l, valid, p.O + (bh * N + (valid ? row : 0)) * D,
-                   p.LSE + bh * N + (valid ? row : 0));
+      const bool issuer = (warp == 4 + 4 * t) && lane == 0;   // of this tile's TMA stores
+      uint8_t* stage = tiles_base + C::kOffStage + t * C::kQBytes;
+      const int bh = item_of(wi).bh, row = tile_row0 + r;
+      if (issuer) bulk_wait_read0();   // the previous item's store has read the staging
+      named_sync(1 + t, 128);
+      stage_row<D>(oreg, true, l, r, stage);
+      if (row < N) p.LSE[(size_t)bh * N + row] = (l > 0.f) ? (m_ref + log2f(l)) * kLn2 : -INFINITY;
+      fence_async_smem();
+      named_sync(1 + t, 128);
+      if (issuer) {
+#pragma unroll
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_store_3d(&p.to, stage + cb * C::kBlockBytes, cb * 64, tile_row0, bh);
+        bulk_commit();
+      }
     }
+    if ((warp == 4 + 4 * t) && lane == 0) bulk_wait_read0();   // staging read before exit
   }
 
   tc_fence_before();
@@ -1043,6 +1122,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
     tc_fence_after();
     tmem_dealloc(tm, 512);
   }
+  // The last CTA to leave resets the queue for the next launch (every CTA
+  // has stopped drawing from it by now).
+  if (threadIdx.x == 0 && atomicAdd(ctas_done, 1u) == gridDim.x - 1) {
+    atomicExch(next_item, 0u);
+    atomicExch(ctas_done, 0u);
+  }
 }
 
 // Dynamic shared memory of one form: control block, alignment slack, tiles.
@@ -1050,8 +1135,13 @@ template <int D, bool kSkip>
 constexpr size_t smem_bytes() {
   return sizeof(Ctl<kSkip>) + 1024 + Cfg<D, kSkip>::kOffEnd;
 }
+template <int D>
+constexpr size_t persist_smem_bytes() {
+  return sizeof(Ctl<false>) + 1024 + PCfg<D>::kOffEnd;
+}
 static_assert(smem_bytes<128, false>() <= 232448 && smem_bytes<128, true>() <= 232448 &&
-                  smem_bytes<64, false>() <= 232448 && smem_bytes<64, true>() <= 232448,
+                  smem_bytes<64, false>() <= 232448 && smem_bytes<64, true>() <= 232448 &&
+                  persist_smem_bytes<128>() <= 232448 && persist_smem_bytes<64>() <= 232448,
               "227 KB of shared memory per CTA");
 
 template <int D>
@@ -1090,8 +1180,10 @@ cudaError_t launch(const Problem& pr) {
                          std::make_pair((const void*)fwd_kernel<D, false, true, false>, smem_skip),
                          std::make_pair((const void*)fwd_kernel<D, false, false, true>, smem_lock),
                          std::make_pair((const void*)fwd_kernel<D, false, true, true>, smem_skip),
-                         std::make_pair((const void*)fwd_persist_kernel<D, false>, smem_lock),
-                         std::make_pair((const void*)fwd_persist_kernel<D, true>, smem_lock)}) {
+                         std::make_pair((const void*)fwd_persist_kernel<D, false>,
+                                        persist_smem_bytes<D>()),
+                         std::make_pair((const void*)fwd_persist_kernel<D, true>,
+                                        persist_smem_bytes<D>())}) {
     const cudaError_t e = set_max_dynamic_smem(fs.first, (int)fs.second);
     if (e != cudaSuccess) return e;
   }
@@ -1112,7 +1204,7 @@ cudaError_t launch(const Problem& pr) {
   const bool skip = !pr.cu && gaps;
   if (!skip && gaps) return cudaErrorInvalidValue;
   if (pr.cu && cap) return cudaErrorInvalidValue;   // not offered for packed batches
-  if (FA_FWD_PERSIST && !pr.cu && !skip) {
+  if (!pr.cu && !skip && pr.N <= FA_FWD_PERSIST_MAXN) {
     // one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -1120,10 +1212,11 @@ cudaError_t launch(const Problem& pr) {
     if (e != cudaSuccess) return e;
     const uint64_t items = BHq * (uint64_t)kp.nblk;
     const dim3 pgrid((unsigned)std::min<uint64_t>(items, (uint64_t)std::max(sms, 1)));
+    const size_t smem_p = persist_smem_bytes<D>();
     if (cap)
-      fwd_persist_kernel<D, true><<<pgrid, kThreads, smem_lock, pr.stream>>>(kp);
+      fwd_persist_kernel<D, true><<<pgrid, kThreads, smem_p, pr.stream>>>(kp);
     else
-      fwd_persist_kernel<D, false><<<pgrid, kThreads, smem_lock, pr.stream>>>(kp);
+      fwd_persist_kernel<D, false><<<pgrid, kThreads, smem_p, pr.stream>>>(kp);
     count_launch();
     return cudaGetLastError();
   }

@@ -79,7 +79,8 @@ const char* fa_status_string(int status);
 /* ABI version: major * 10000 + minor * 100 + patch. */
 int fa_version(void);
 
-/* Bytes of workspace fa_fwd needs: the 256-byte error-word block. */
+/* Bytes of workspace fa_fwd needs: the 256-byte error-word block (the
+ * backward's workspace starts with the same block and may serve both). */
 size_t fa_fwd_workspace_size(void);
 
 /* Bytes of workspace fa_bwd needs: the error-word block, D and the
@@ -93,8 +94,12 @@ size_t fa_bwd_workspace_size(int B, int Hq, int N, int d);
  *   Q [B,Hq,N,d], K and V [B,Hkv,N,d] (dtype); O [B,Hq,N,d] (dtype);
  *   LSE [B,Hq,N] float; scale: the softmax scale (1/sqrt(d) in the pages);
  *   causal: 0 or 1; block_mask: NULL or device uint8 [nb*nb];
- *   workspace: >= fa_fwd_workspace_size() bytes, device, zeroed once before
- *   first use (it then holds the error word, which fa_get_device_error clears).
+ *   workspace: >= fa_fwd_workspace_size() bytes, device, its first 256 bytes
+ *   zeroed once before first use. That block holds the error word (which
+ *   fa_get_device_error clears) and, for the persistent form of the kernel, a
+ *   work-queue counter that each launch leaves at zero again. A workspace
+ *   serves one launch at a time: launches that may overlap on the GPU need
+ *   workspaces of their own.
  * Supported: d in {16, 32, 64, 128}; Hq % Hkv == 0; N >= 0, B >= 0 (an empty
  * problem launches nothing and returns FA_OK).
  */
