@@ -156,6 +156,18 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
+// mbar_wait with the checks in the other order: a phase that has already
+// completed is taken before the abort flag is read, so the fast path is one
+// shared-memory operation instead of two. Used where the waits sit on the
+// MMA issue chain (the forward kernels: measured 5-7 % faster on B200; the
+// backward main kernel measured 1 % slower with it and keeps mbar_wait).
+__device__ __forceinline__ bool mbar_wait_ready_first(uint64_t* bar, uint32_t parity,
+                                                      const Guard& g,
+                                                      long long limit = kWaitLimitCycles) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait(bar, parity, g, limit);
+}
+
 // Test hook of the bounded-wait contract: when stall_cycles > 0 the caller
 // waits on `never`, a barrier initialised with one expected arrival that
 // nothing ever signals, with that short limit. The wait runs out and takes

@@ -511,7 +511,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       int issued = pre_loads;
       for (int n = pre_loads; n < 2 * T; ++n) {
         const int s = ring_slot<kSlots>(n);
-        if (n >= kSlots && !mbar_wait(&ctl.kv_empty[s], ring_phase<kSlots>(n - kSlots), g)) break;
+        if (n >= kSlots && !mbar_wait_ready_first(&ctl.kv_empty[s], ring_phase<kSlots>(n - kSlots), g)) break;
         const int kb = tile_of(n >> 1);
         const CUtensorMap* m = (n & 1) ? &p.tv : &p.tk;
         mbar_expect_tx(&ctl.kv_full[s], C::kTileBytes);
@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
       const uint32_t kva = smem_u32(tiles_base + C::kOffKV);
       auto slot_addr = [&](int n) { return kva + ring_slot<kSlots>(n) * C::kTileBytes; };
       auto wait_tile = [&](int n) {
-        return mbar_wait(&ctl.kv_full[ring_slot<kSlots>(n)], ring_phase<kSlots>(n), g);
+        return mbar_wait_ready_first(&ctl.kv_full[ring_slot<kSlots>(n)], ring_phase<kSlots>(n), g);
       };
       auto release_tile = [&](int n) { mma_commit(&ctl.kv_empty[ring_slot<kSlots>(n)]); };
       // S_t = Q_t K_j^T
@@ -570,7 +570,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         const int nl0 = ctl.nlive[0], nl1 = ctl.nlive[1];
         int n0 = 0, n1 = 0;
         int live_next = T > 0 ? (~ctl.l.dead[0] & 3) : 0;
-        bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait(&ctl.q_full, 0, g) &&
+        bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait_ready_first(&ctl.q_full, 0, g) &&
                   wait_tile(0);
         if (ok) {
           tc_fence_after();
@@ -590,10 +590,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           live_next = more ? (~ctl.l.dead[j + 1] & 3) : 0;
           if (!(ok = wait_tile(2 * j + 1))) break;
           if (live_cur & 1) {
-            if (!(ok = mbar_wait(&ctl.p_half[0], n0 & 1, g))) break;
+            if (!(ok = mbar_wait_ready_first(&ctl.p_half[0], n0 & 1, g))) break;
             tc_fence_after();
             issue_pv(0, j, n0 > 0, 0);
-            if (!(ok = mbar_wait(&ctl.p_full[0], n0 & 1, g))) break;
+            if (!(ok = mbar_wait_ready_first(&ctl.p_full[0], n0 & 1, g))) break;
             tc_fence_after();
             issue_pv(0, j, n0 > 0, 1);
             if (++n0 == nl0) mma_commit(&ctl.o_ready[0]);
@@ -607,10 +607,10 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
             }
           }
           if (live_cur & 2) {
-            if (!(ok = mbar_wait(&ctl.p_half[1], n1 & 1, g))) break;
+            if (!(ok = mbar_wait_ready_first(&ctl.p_half[1], n1 & 1, g))) break;
             tc_fence_after();
             issue_pv(1, j, n1 > 0, 0);
-            if (!(ok = mbar_wait(&ctl.p_full[1], n1 & 1, g))) break;
+            if (!(ok = mbar_wait_ready_first(&ctl.p_full[1], n1 & 1, g))) break;
             tc_fence_after();
             issue_pv(1, j, n1 > 0, 1);
             if (++n1 == nl1) mma_commit(&ctl.o_ready[1]);
@@ -628,7 +628,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
         if (n0 != nl0 || nl0 == 0) mma_commit(&ctl.o_ready[0]);
         if (n1 != nl1 || nl1 == 0) mma_commit(&ctl.o_ready[1]);
       } else {
-        bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait(&ctl.q_full, 0, g) &&
+        bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait_ready_first(&ctl.q_full, 0, g) &&
                   wait_tile(0);
         if (ok) {
           tc_fence_after();
@@ -639,25 +639,28 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
           release_tile(0);
         }
         for (int j = 0; ok && j < T; ++j) {
-          if (!(ok = wait_tile(2 * j + 1) && mbar_wait(&ctl.p_half[0], j & 1, g))) break;
+          const bool more = j + 1 < T;
+          // V_j and K_{j+1} (long landed as a rule) are checked here, while P
+          // is still being computed, so that nothing but the P signals sits
+          // between a tile's last P V and its next S.
+          if (!(ok = wait_tile(2 * j + 1) && (!more || wait_tile(2 * j + 2)) &&
+                     mbar_wait_ready_first(&ctl.p_half[0], j & 1, g)))
+            break;
           tc_fence_after();
           issue_pv(0, j, j > 0, 0);
-          if (!(ok = mbar_wait(&ctl.p_full[0], j & 1, g))) break;
+          if (!(ok = mbar_wait_ready_first(&ctl.p_full[0], j & 1, g))) break;
           tc_fence_after();
           issue_pv(0, j, j > 0, 1);
-          const bool more = j + 1 < T;
           // the last P V of a query tile: its epilogue may start
           if (!more) mma_commit(&ctl.o_ready[0]);
           if (more) {
-            if (!(ok = wait_tile(2 * j + 2))) break;
-            tc_fence_after();
             issue_s(0, j + 1);
             mma_commit(&ctl.s_full[0]);
           }
-          if (!(ok = mbar_wait(&ctl.p_half[1], j & 1, g))) break;
+          if (!(ok = mbar_wait_ready_first(&ctl.p_half[1], j & 1, g))) break;
           tc_fence_after();
           issue_pv(1, j, j > 0, 0);
-          if (!(ok = mbar_wait(&ctl.p_full[1], j & 1, g))) break;
+          if (!(ok = mbar_wait_ready_first(&ctl.p_full[1], j & 1, g))) break;
           tc_fence_after();
           issue_pv(1, j, j > 0, 1);
           if (!more) mma_commit(&ctl.o_ready[1]);
@@ -699,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     int it = kSkip ? t : 0;
     for (; it < it_end; it += kStep) {
       const int n = kSkip ? (it >> 1) : it;   // tiles of this query tile so far
-      if (!mbar_wait(&ctl.s_full[t], n & 1, g)) break;
+      if (!mbar_wait_ready_first(&ctl.s_full[t], n & 1, g)) break;
       tc_fence_after();
       uint32_t sr[128];
       tmem_ld128(sreg, sr);
@@ -747,12 +750,12 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     if (have_o) {
       // this query tile's last P V has completed (its S MMAs, which read the
       // Q buffer, came before it)
-      mbar_wait(&ctl.o_ready[t], 0, g);
+      mbar_wait_ready_first(&ctl.o_ready[t], 0, g);
       tc_fence_after();
     } else {
       // no MMA read this tile's Q buffer, but its load may still be landing:
       // wait for it before the buffer is reused for the output
-      mbar_wait(&ctl.q_full, 0, g);
+      mbar_wait_ready_first(&ctl.q_full, 0, g);
     }
     const bool valid = row < N;
     if constexpr (!kVarlen) {
@@ -909,7 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
         // the next item for this CTA (or -1: the queue is empty)
         const int slot = k % kItemRing;
         if (k >= kItemRing &&
-            !(ok = mbar_wait(&ctl.item_empty[slot], ((k / kItemRing) - 1) & 1, g)))
+            !(ok = mbar_wait_ready_first(&ctl.item_empty[slot], ((k / kItemRing) - 1) & 1, g)))
           break;
         const unsigned w = atomicAdd(next_item, 1u);
         const int wi = (w < (unsigned)W) ? (int)w : -1;
@@ -919,7 +922,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
         const Item it = item_of(wi);
         // Q tile t once the previous item's last S_t has read the buffer
         for (int t = 0; ok && t < 2; ++t) {
-          if (qi[t] > 0 && !(ok = mbar_wait(&ctl.qt_empty[t], (qi[t] - 1) & 1, g))) break;
+          if (qi[t] > 0 && !(ok = mbar_wait_ready_first(&ctl.qt_empty[t], (qi[t] - 1) & 1, g))) break;
           mbar_expect_tx(&ctl.qt_full[t], C::kQBytes);
           for (int cb = 0; cb < C::kColBlocks; ++cb)
             tma_load_3d(tiles_base + C::kOffQ + t * C::kQBytes + cb * C::kBlockBytes, &p.tq,
@@ -928,7 +931,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
         }
         for (int j = 0; ok && j < 2 * it.T; ++j, ++n) {
           const int s = ring_slot<kSlots>(n);
-          if (n >= kSlots && !(ok = mbar_wait(&ctl.kv_empty[s], ring_phase<kSlots>(n - kSlots), g)))
+          if (n >= kSlots && !(ok = mbar_wait_ready_first(&ctl.kv_empty[s], ring_phase<kSlots>(n - kSlots), g)))
             break;
           mbar_expect_tx(&ctl.kv_full[s], C::kTileBytes);
           for (int cb = 0; cb < C::kColBlocks; ++cb)
@@ -954,7 +957,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
       const uint32_t kva = smem_u32(tiles_base + C::kOffKV);
       auto slot_addr = [&](int n) { return kva + ring_slot<kSlots>(n) * C::kTileBytes; };
       auto wait_tile = [&](int n) {
-        return mbar_wait(&ctl.kv_full[ring_slot<kSlots>(n)], ring_phase<kSlots>(n), g);
+        return mbar_wait_ready_first(&ctl.kv_full[ring_slot<kSlots>(n)], ring_phase<kSlots>(n), g);
       };
       auto release_tile = [&](int n) { mma_commit(&ctl.kv_empty[ring_slot<kSlots>(n)]); };
       // S_t = Q_t K^T with K the ring tile n
@@ -982,14 +985,14 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
       int n = 0, nt = 0;   // ring tiles and softmax tiles so far
       for (int k = 0; ok; ++k) {
         const int slot = k % kItemRing;
-        if (!(ok = mbar_wait(&ctl.item_full[slot], (k / kItemRing) & 1, g))) break;
+        if (!(ok = mbar_wait_ready_first(&ctl.item_full[slot], (k / kItemRing) & 1, g))) break;
         const int wi = ctl.item_id[slot];
         mbar_arrive(&ctl.item_empty[slot]);
         if (wi < 0) break;
         const int T = item_of(wi).T;
         // K_j is ring tile n + 2j, V_j is n + 2j + 1
         for (int t = 0; t < 2; ++t) {
-          if (!(ok = mbar_wait(&ctl.qt_full[t], k & 1, g) && wait_tile(n))) break;
+          if (!(ok = mbar_wait_ready_first(&ctl.qt_full[t], k & 1, g) && wait_tile(n))) break;
           tc_fence_after();
           issue_s(t, n);
           mma_commit(&ctl.s_full[t]);
@@ -1000,24 +1003,25 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
         for (int j = 0; ok && j < T; ++j) {
           const uint32_t ph = (nt + j) & 1;
           const bool more = j + 1 < T;
-          if (!(ok = wait_tile(n + 2 * j + 1) && mbar_wait(&ctl.p_half[0], ph, g))) break;
+          // (as in the one-item form: the next K tile is checked before P)
+          if (!(ok = wait_tile(n + 2 * j + 1) && (!more || wait_tile(n + 2 * j + 2)) &&
+                     mbar_wait_ready_first(&ctl.p_half[0], ph, g)))
+            break;
           tc_fence_after();
           issue_pv(0, n + 2 * j + 1, j > 0, 0);
-          if (!(ok = mbar_wait(&ctl.p_full[0], ph, g))) break;
+          if (!(ok = mbar_wait_ready_first(&ctl.p_full[0], ph, g))) break;
           tc_fence_after();
           issue_pv(0, n + 2 * j + 1, j > 0, 1);
           if (!more) mma_commit(&ctl.o_ready[0]);
           if (more) {
-            if (!(ok = wait_tile(n + 2 * j + 2))) break;
-            tc_fence_after();
             issue_s(0, n + 2 * j + 2);
             mma_commit(&ctl.s_full[0]);
             if (j + 2 == T) mma_commit(&ctl.qt_empty[0]);
           }
-          if (!(ok = mbar_wait(&ctl.p_half[1], ph, g))) break;
+          if (!(ok = mbar_wait_ready_first(&ctl.p_half[1], ph, g))) break;
           tc_fence_after();
           issue_pv(1, n + 2 * j + 1, j > 0, 0);
-          if (!(ok = mbar_wait(&ctl.p_full[1], ph, g))) break;
+          if (!(ok = mbar_wait_ready_first(&ctl.p_full[1], ph, g))) break;
           tc_fence_after();
           issue_pv(1, n + 2 * j + 1, j > 0, 1);
           if (!more) mma_commit(&ctl.o_ready[1]);
@@ -1048,7 +1052,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
     int nt = 0;
     for (int k = 0; ok; ++k) {
       const int slot = k % kItemRing;
-      if (!(ok = mbar_wait(&ctl.item_full[slot], (k / kItemRing) & 1, g))) break;
+      if (!(ok = mbar_wait_ready_first(&ctl.item_full[slot], (k / kItemRing) & 1, g))) break;
       const int wi = ctl.item_id[slot];
       __syncwarp();
       if (lane == 0) mbar_arrive(&ctl.item_empty[slot]);
@@ -1063,7 +1067,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
       }
       float m_ref = -INFINITY, l = 0.f;
       for (int j = 0; j < T; ++j) {
-        if (!(ok = mbar_wait(&ctl.s_full[t], (nt + j) & 1, g))) break;
+        if (!(ok = mbar_wait_ready_first(&ctl.s_full[t], (nt + j) & 1, g))) break;
         tc_fence_after();
         uint32_t sr[128];
         tmem_ld128(sreg, sr);
@@ -1095,7 +1099,7 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
       if (!ok) break;
       nt += T;
       // epilogue of this item: the last P V of this query tile has completed
-      if (!(ok = mbar_wait(&ctl.o_ready[t], k & 1, g))) break;
+      if (!(ok = mbar_wait_ready_first(&ctl.o_ready[t], k & 1, g))) break;
       tc_fence_after();
       const bool issuer = (warp == 4 + 4 * t) && lane == 0;   // of this tile's TMA stores
       uint8_t* stage = tiles_base + C::kOffStage + t * C::kQBytes;
