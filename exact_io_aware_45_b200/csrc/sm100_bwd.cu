@@ -353,66 +353,68 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       constexpr uint32_t idSP = idesc_bf16(kBN, MQ, false, false);   // K-major A and B
       constexpr uint32_t idKV = idesc_bf16(kBN, D, false, true);     // B MN-major
       constexpr uint32_t idQ = idesc_bf16(128, 64, true, true);      // both MN-major
+      // Base descriptors, built once (K-major and MN-major readings of K, V,
+      // the Q / dO ring and the dS^T buffers); each operand below is one of
+      // them plus a byte offset (sdesc_at).
       const uint32_t ka = smem_u32(base + C::kOffK), va = smem_u32(base + C::kOffV);
       const uint32_t qa = smem_u32(base + C::kOffQ), da = smem_u32(base + C::kOffDO);
       const uint32_t dsa = smem_u32(base + C::kOffDS);
-      auto qstage = [&](int i) { return qa + (i % C::kStages) * C::kQBytes; };
-      auto dostage = [&](int i) { return da + (i % C::kStages) * C::kQBytes; };
-      auto dsbuf = [&](int i) { return dsa + (i & 1) * C::kDSBytes; };
+      const uint64_t dK_k = sdesc_sw128(ka, 16, 1024), dV_k = sdesc_sw128(va, 16, 1024);
+      const uint64_t dQ_k = sdesc_sw128(qa, 16, 1024), dO_k = sdesc_sw128(da, 16, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(qa, C::kQBlock, 1024);
+      const uint64_t dO_mn = sdesc_sw128(da, C::kQBlock, 1024);
+      const uint64_t dS_k = sdesc_sw128(dsa, 16, 1024);
+      const uint64_t dK_mn = sdesc_sw128(ka, kBN * 128, 1024);
+      const uint64_t dS_mn = sdesc_sw128(dsa, kBN * 128, 1024);
+      auto qoff = [&](int i) { return (uint32_t)((i % C::kStages) * C::kQBytes); };
+      auto dsoff = [&](int i) { return (uint32_t)((i & 1) * C::kDSBytes); };
       auto issue_s = [&](int i) {   // S^T = K Q_i^T
-        const uint32_t qs = qstage(i);
+        const uint64_t dq = sdesc_at(dQ_k, qoff(i));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tm + s_col(i),
-                 sdesc_sw128(ka + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(qs + (kk >> 2) * C::kQBlock + (kk & 3) * 32, 16, 1024), idSP,
-                 kk > 0);
+          mma_ss(tm + s_col(i), sdesc_at(dK_k, (kk >> 2) * (kBN * 128) + (kk & 3) * 32),
+                 sdesc_at(dq, (kk >> 2) * C::kQBlock + (kk & 3) * 32), idSP, kk > 0);
       };
       auto issue_dp = [&](int i) {  // dP^T = V dO_i^T
-        const uint32_t ds_ = dostage(i);
+        const uint64_t ddo = sdesc_at(dO_k, qoff(i));
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(tm + dp_col(i),
-                 sdesc_sw128(va + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
-                 sdesc_sw128(ds_ + (kk >> 2) * C::kQBlock + (kk & 3) * 32, 16, 1024), idSP,
-                 kk > 0);
+          mma_ss(tm + dp_col(i), sdesc_at(dV_k, (kk >> 2) * (kBN * 128) + (kk & 3) * 32),
+                 sdesc_at(ddo, (kk >> 2) * C::kQBlock + (kk & 3) * 32), idSP, kk > 0);
       };
       // dV += P^T dO_i and dK += dS^T Q_i over the query columns the softmax
       // warps finished in chunk step `st` (32-column chunk cc = h * kChunks + st
       // of each column half h; 16-query k-steps 2cc and 2cc + 1).
       auto issue_dv = [&](int i, int st) {  // P^T bf16 in the S columns
-        const uint32_t dos = dostage(i);
+        const uint64_t ddo = sdesc_at(dO_mn, qoff(i));
 #pragma unroll
         for (int h = 0; h < C::kColHalves; ++h)
 #pragma unroll
           for (int k2 = 0; k2 < 2; ++k2) {
             const int kk = 2 * (h * kChunks + st) + k2;
             mma_ts(tm + C::kDV, tm + s_col(i) + (kk >> 1) * 32 + (kk & 1) * 8,
-                   sdesc_sw128(dos + kk * 2048, C::kQBlock, 1024), idKV, (i > 0 || kk > 0));
+                   sdesc_at(ddo, kk * 2048), idKV, (i > 0 || kk > 0));
           }
       };
       auto issue_dk = [&](int i, int st) {
-        const uint32_t qs = qstage(i), dsb = dsbuf(i);
+        const uint64_t dq = sdesc_at(dQ_mn, qoff(i)), ds = sdesc_at(dS_k, dsoff(i));
 #pragma unroll
         for (int h = 0; h < C::kColHalves; ++h)
 #pragma unroll
           for (int k2 = 0; k2 < 2; ++k2) {
             const int kk = 2 * (h * kChunks + st) + k2;
-            mma_ss(tm + C::kDK,
-                   sdesc_sw128(dsb + (kk >> 2) * (kBN * 128) + (kk & 3) * 32, 16, 1024),
-                   sdesc_sw128(qs + kk * 2048, C::kQBlock, 1024), idKV, (i > 0 || kk > 0));
+            mma_ss(tm + C::kDK, sdesc_at(ds, (kk >> 2) * (kBN * 128) + (kk & 3) * 32),
+                   sdesc_at(dq, kk * 2048), idKV, (i > 0 || kk > 0));
           }
       };
       auto issue_dq = [&](int i) {  // dQ_i^T = K^T dS_i^T (d = 128) or dQ_i = dS_i K (d = 64)
-        const uint32_t dsb = dsbuf(i);
+        const uint64_t ds = sdesc_at(dS_mn, dsoff(i));
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk) {
           if constexpr (D == 128)
-            mma_ss(tm + dq_col(i), sdesc_sw128(ka + kk * 2048, kBN * 128, 1024),
-                   sdesc_sw128(dsb + kk * 2048, kBN * 128, 1024), idQ, kk > 0);
+            mma_ss(tm + dq_col(i), sdesc_at(dK_mn, kk * 2048), sdesc_at(ds, kk * 2048), idQ, kk > 0);
           else
-            mma_ss(tm + dq_col(i), sdesc_sw128(dsb + kk * 2048, kBN * 128, 1024),
-                   sdesc_sw128(ka + kk * 2048, kBN * 128, 1024), idQ, kk > 0);
+            mma_ss(tm + dq_col(i), sdesc_at(ds, kk * 2048), sdesc_at(dK_mn, kk * 2048), idQ, kk > 0);
         }
       };
       auto wait_q = [&](int i) {

@@ -529,6 +529,13 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// Descriptor of the operand `off` bytes (a multiple of 16) past the one `d`
+// describes, with the same layout: the start-address field holds the address
+// / 16 in its low 14 bits and shared memory ends below 256 KB, so adding
+// off / 16 never carries out of the field. Cheaper than rebuilding the
+// descriptor on an MMA issue path.
+__device__ __forceinline__ uint64_t sdesc_at(uint64_t d, uint32_t off) { return d + (off >> 4); }
+
 // Instruction descriptor, kind::f16: bf16 x bf16 -> f32, dense.
 // a_mn / b_mn: operand is MN-major (else K-major).
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn) {

@@ -532,32 +532,36 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_kernel(const __grid_constant_
     if (lane == 0 && T > 0) {
       constexpr uint32_t idS = idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t idO = idesc_bf16(kBM, D, false, true);
-      const uint32_t qa = smem_u32(tiles_base + C::kOffQ);
-      const uint32_t kva = smem_u32(tiles_base + C::kOffKV);
-      auto slot_addr = [&](int n) { return kva + ring_slot<kSlots>(n) * C::kTileBytes; };
+      // Base descriptors, built once: Q tile 0 (tile 1 follows it), ring slot
+      // 0 read as a K tile (K-major) and as a V tile (MN-major); every MMA
+      // operand below is one of them plus a byte offset (sdesc_at), which
+      // keeps the issue path after each P signal short.
+      const uint64_t dq0 = sdesc_sw128(smem_u32(tiles_base + C::kOffQ), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(tiles_base + C::kOffKV), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(tiles_base + C::kOffKV), C::kBlockBytes, 1024);
       auto wait_tile = [&](int n) {
         return mbar_wait_ready_first(&ctl.kv_full[ring_slot<kSlots>(n)], ring_phase<kSlots>(n), g);
       };
       auto release_tile = [&](int n) { mma_commit(&ctl.kv_empty[ring_slot<kSlots>(n)]); };
       // S_t = Q_t K_j^T
       auto issue_s = [&](int t, int j) {
-        const uint32_t qt = qa + t * C::kQBytes, kt = slot_addr(2 * j);
+        const uint64_t dq = sdesc_at(dq0, t * C::kQBytes);
+        const uint64_t dk = sdesc_at(dk0, ring_slot<kSlots>(2 * j) * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
-          mma_ss(tm + (t ? C::kS1 : C::kS0), sdesc_sw128(qt + off, 16, 1024),
-                 sdesc_sw128(kt + off, 16, 1024), idS, kk > 0);
+          mma_ss(tm + (t ? C::kS1 : C::kS0), sdesc_at(dq, off), sdesc_at(dk, off), idS, kk > 0);
         }
       };
       // O_t += P_t V_j over keys 64*hf .. 64*hf+63 of the tile.
       auto issue_pv = [&](int t, int j, bool acc, int hf) {
-        const uint32_t vt = slot_addr(2 * j + 1);
+        const uint64_t dv = sdesc_at(dv0, ring_slot<kSlots>(2 * j + 1) * C::kTileBytes);
         const uint32_t pt = tm + (t ? C::kS1 : C::kS0) + C::kPOff;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int kk = 4 * hf + k4;
-          mma_ts(tm + (t ? C::kO1 : C::kO0), pt + kk * 8,
-                 sdesc_sw128(vt + kk * 16 * 128, C::kBlockBytes, 1024), idO, (acc || kk > 0));
+          mma_ts(tm + (t ? C::kO1 : C::kO0), pt + kk * 8, sdesc_at(dv, kk * 16 * 128), idO,
+                 (acc || kk > 0));
         }
       };
       if constexpr (kSkip) {
@@ -953,32 +957,33 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t idO = idesc_bf16(kBM, D, false, true);
-      const uint32_t qa = smem_u32(tiles_base + C::kOffQ);
-      const uint32_t kva = smem_u32(tiles_base + C::kOffKV);
-      auto slot_addr = [&](int n) { return kva + ring_slot<kSlots>(n) * C::kTileBytes; };
+      // base descriptors, as in the one-item form
+      const uint64_t dq0 = sdesc_sw128(smem_u32(tiles_base + C::kOffQ), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(tiles_base + C::kOffKV), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(tiles_base + C::kOffKV), C::kBlockBytes, 1024);
       auto wait_tile = [&](int n) {
         return mbar_wait_ready_first(&ctl.kv_full[ring_slot<kSlots>(n)], ring_phase<kSlots>(n), g);
       };
       auto release_tile = [&](int n) { mma_commit(&ctl.kv_empty[ring_slot<kSlots>(n)]); };
       // S_t = Q_t K^T with K the ring tile n
       auto issue_s = [&](int t, int n) {
-        const uint32_t qt = qa + t * C::kQBytes, kt = slot_addr(n);
+        const uint64_t dq = sdesc_at(dq0, t * C::kQBytes);
+        const uint64_t dk = sdesc_at(dk0, ring_slot<kSlots>(n) * C::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
-          mma_ss(tm + (t ? C::kS1 : C::kS0), sdesc_sw128(qt + off, 16, 1024),
-                 sdesc_sw128(kt + off, 16, 1024), idS, kk > 0);
+          mma_ss(tm + (t ? C::kS1 : C::kS0), sdesc_at(dq, off), sdesc_at(dk, off), idS, kk > 0);
         }
       };
       // O_t += P_t V over keys 64*hf .. 64*hf+63 of the ring tile n (a V tile)
       auto issue_pv = [&](int t, int n, bool acc, int hf) {
-        const uint32_t vt = slot_addr(n);
+        const uint64_t dv = sdesc_at(dv0, ring_slot<kSlots>(n) * C::kTileBytes);
         const uint32_t pt = tm + (t ? C::kS1 : C::kS0) + C::kPOff;
 #pragma unroll
         for (int k4 = 0; k4 < 4; ++k4) {
           const int kk = 4 * hf + k4;
-          mma_ts(tm + (t ? C::kO1 : C::kO0), pt + kk * 8,
-                 sdesc_sw128(vt + kk * 16 * 128, C::kBlockBytes, 1024), idO, (acc || kk > 0));
+          mma_ts(tm + (t ? C::kO1 : C::kO0), pt + kk * 8, sdesc_at(dv, kk * 16 * 128), idO,
+                 (acc || kk > 0));
         }
       };
       bool ok = injected_stall(&ctl.never, p.stall, g);
