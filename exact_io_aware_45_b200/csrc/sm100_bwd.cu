@@ -417,8 +417,10 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
             mma_ss(tm + dq_col(i), sdesc_at(ds, kk * 2048), sdesc_at(dK_mn, kk * 2048), idQ, kk > 0);
         }
       };
+      // (normally landed long before: the phase is tested before the abort
+      // flag is read)
       auto wait_q = [&](int i) {
-        return mbar_wait(&ctl.qdo_full[i % C::kStages], (i / C::kStages) & 1, g);
+        return mbar_wait_ready_first(&ctl.qdo_full[i % C::kStages], (i / C::kStages) & 1, g);
       };
       bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait(&ctl.kv_full, 0, g) &&
                 wait_q(0);
@@ -517,7 +519,7 @@ __global__ void __launch_bounds__(Cfg<D>::kThreads, 1) bwd_kernel(const __grid_c
       const bool spok = C::kDbl ? mbar_wait(&ctl.sp_full[i & 1], (i >> 1) & 1, g)
                                 : mbar_wait(&ctl.sp_full[0], i & 1, g);
       if (!spok) break;
-      if (!mbar_wait(&ctl.qdo_full[s], (i / C::kStages) & 1, g)) break;
+      if (!mbar_wait_ready_first(&ctl.qdo_full[s], (i / C::kStages) & 1, g)) break;
       tc_fence_after();
       const int q0 = item_q0(i);
       const bool need_mask = !(ctl.qtiles[i % nq] & kFullBit);

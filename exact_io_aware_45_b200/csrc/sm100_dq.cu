@@ -198,17 +198,18 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
     if (lane == 0 && T > 0) {
       constexpr uint32_t idS = idesc_bf16(kBM, kBN, false, false);
       constexpr uint32_t idQ = idesc_bf16(kBM, D, false, true);
-      const uint32_t qa = smem_u32(tiles_base + C::kOffQ);
-      const uint32_t da = smem_u32(tiles_base + C::kOffDO);
-      const uint32_t ka = smem_u32(tiles_base + C::kOffK);
-      const uint32_t va = smem_u32(tiles_base + C::kOffV);
+      // base descriptors, built once; each operand is one plus a byte offset
+      const uint64_t dQd = sdesc_sw128(smem_u32(tiles_base + C::kOffQ), 16, 1024);
+      const uint64_t dOd = sdesc_sw128(smem_u32(tiles_base + C::kOffDO), 16, 1024);
+      const uint64_t dKd = sdesc_sw128(smem_u32(tiles_base + C::kOffK), 16, 1024);
+      const uint64_t dVd = sdesc_sw128(smem_u32(tiles_base + C::kOffV), 16, 1024);
+      const uint64_t dKn = sdesc_sw128(smem_u32(tiles_base + C::kOffK), C::kBlockBytes, 1024);
       // X Y^T over d for X in {Q, dO} (128 x d) and Y in {K_j, V_j} (128 x d)
-      auto issue_xy = [&](uint32_t dst, uint32_t xa, uint32_t ya) {
+      auto issue_xy = [&](uint32_t dst, uint64_t xd, uint64_t yd) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
-          mma_ss(tm + dst, sdesc_sw128(xa + off, 16, 1024), sdesc_sw128(ya + off, 16, 1024), idS,
-                 kk > 0);
+          mma_ss(tm + dst, sdesc_at(xd, off), sdesc_at(yd, off), idS, kk > 0);
         }
       };
       bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait(&ctl.q_full, 0, g);
@@ -216,17 +217,18 @@ __global__ void __launch_bounds__(kThreads, 1) dq_kernel(const __grid_constant__
         const int s = j % C::kStages;
         if (!(ok = mbar_wait(&ctl.kv_full[s], (j / C::kStages) & 1, g))) break;
         tc_fence_after();
-        const uint32_t kt = ka + s * C::kTileBytes, vt = va + s * C::kTileBytes;
-        issue_xy(C::kS, qa, kt);    // S = Q K_j^T
-        issue_xy(C::kDP, da, vt);   // dP = dO V_j^T
+        const uint32_t so = s * C::kTileBytes;
+        issue_xy(C::kS, dQd, sdesc_at(dKd, so));    // S = Q K_j^T
+        issue_xy(C::kDP, dOd, sdesc_at(dVd, so));   // dP = dO V_j^T
         mma_commit(&ctl.sp_full);
         if (!(ok = mbar_wait(&ctl.ds_ready, j & 1, g))) break;
         tc_fence_after();
         // dQ += dS K_j (dS bf16 pairs in S's first 64 columns; K_j N-major)
+        const uint64_t kn = sdesc_at(dKn, so);
 #pragma unroll
         for (int kk = 0; kk < kBN / 16; ++kk)
-          mma_ts(tm + C::kDQ, tm + C::kS + kk * 8,
-                 sdesc_sw128(kt + kk * 16 * 128, C::kBlockBytes, 1024), idQ, (j > 0 || kk > 0));
+          mma_ts(tm + C::kDQ, tm + C::kS + kk * 8, sdesc_at(kn, kk * 16 * 128), idQ,
+                 (j > 0 || kk > 0));
         mma_commit(&ctl.kv_empty[s]);
       }
       mma_commit(&ctl.dq_done);

@@ -96,3 +96,28 @@ def test_reference_arm_forward_only_workload():
     assert "forward+backward" not in d["cpu_baseline"]["sample"]
     flops = 2 * 4 * 32 * 512 * 512
     assert abs(d["value"] - flops / (2 * d["ms_per_step"] / 1e3) / 1e12) <= 1e-9 * d["value"]
+
+
+def test_peak_choice_follows_the_timed_region():
+    """The roofline compares with the burst bf16 peak for a short timed region
+    and with the sustained one once the region is long enough to run under the
+    power cap, or its clock record shows the cap holding the clock down; both
+    fractions are always reported."""
+    import bench
+    peaks = {"bf16_tflops": 1669.2, "bf16_tflops_sustained": 1401.3}
+    free = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": []}
+    capped = {"sm_mhz": 1770.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    flag_only = {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0, "reasons": ["sw_power_cap"]}
+    assert bench.select_bf16_peak(peaks, "measured", 50.0, free)[0] == 1669.2
+    assert bench.select_bf16_peak(peaks, "measured", 50.0, flag_only)[0] == 1669.2
+    assert bench.select_bf16_peak(peaks, "measured", 50.0, capped)[0] == 1401.3
+    assert bench.select_bf16_peak(peaks, "measured", 500.0, free)[0] == 1401.3
+    # no sustained figure: always the burst one
+    assert bench.select_bf16_peak({"bf16_tflops": 1669.2}, "measured", 500.0, capped)[0] == 1669.2
+    assert bench.select_bf16_peak(None, "fallback", 500.0, capped)[0] == bench.FALLBACK_PEAK_TFLOPS
+    roof = bench.tensor_roofline("bwd_main", 800.0,
+                                 bench.select_bf16_peak(peaks, "measured", 500.0, free), None)
+    assert abs(roof["frac"] - 800.0 / 1401.3) < 1e-12
+    assert abs(roof["frac_of_burst"] - 800.0 / 1669.2) < 1e-12
+    assert abs(roof["frac_of_sustained"] - 800.0 / 1401.3) < 1e-12
+    assert "sustained" in roof["peak_kind"]
