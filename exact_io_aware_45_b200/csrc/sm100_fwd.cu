@@ -282,19 +282,24 @@ template <int D>
 __device__ __forceinline__ void stage_row(uint32_t oreg, bool have_o, float l, int r,
                                           uint8_t* stage) {
   const float inv = (l > 0.f) ? 1.f / l : 0.f;
+  // the whole row in one TMEM round trip (the score registers are free here)
+  uint32_t o[D];
+  if (have_o) {
+    if constexpr (D == 128)
+      tmem_ld128(oreg, o);
+    else
+      tmem_ld64(oreg, o);
+  } else {
+#pragma unroll
+    for (int i = 0; i < D; ++i) o[i] = 0u;
+  }
 #pragma unroll
   for (int cc = 0; cc < D / 32; ++cc) {
-    uint32_t o[32];
-    if (have_o) {
-      tmem_ld32(oreg + cc * 32, o);
-    } else {
-#pragma unroll
-      for (int i = 0; i < 32; ++i) o[i] = 0u;
-    }
     uint32_t w[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i)
-      w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+      w[i] = pack_bf16(__uint_as_float(o[32 * cc + 2 * i]) * inv,
+                       __uint_as_float(o[32 * cc + 2 * i + 1]) * inv);
     uint8_t* rowp = stage + (cc >> 1) * 16384 + r * 128;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
