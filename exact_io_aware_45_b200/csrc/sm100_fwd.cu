@@ -84,6 +84,11 @@ constexpr int kMaxSlots = 10;     // most K/V ring slots of any form
 // measured on B200, the persistent form is 1-13% faster up to N = 4096 (the
 // fixed cost per item matters most there) and 3-6% slower at 8K-16K (its
 // steady state is a little slower). 0: never persistent.
+// Block-sparse launches (a block mask given) run the split form: bit 0 at
+// d = 64, bit 1 at d = 128; otherwise the paired skipping form.
+#ifndef FA_FWD_SPLIT
+#define FA_FWD_SPLIT 3
+#endif
 #ifndef FA_FWD_PERSIST_MAXN
 #define FA_FWD_PERSIST_MAXN 4096
 #endif
@@ -1144,10 +1149,337 @@ __global__ void __launch_bounds__(kThreads, 1) fwd_persist_kernel(const __grid_c
   }
 }
 
+// Split form, for block-sparse launches: one 128-row query tile per CTA,
+// whose visible key tiles (its list L, in increasing order) are dealt to the
+// two softmax warpgroups in turn: stream 0 takes L[0], L[2], ..., stream 1
+// L[1], L[3], .... Both streams read the one Q tile; each keeps its own
+// online-softmax state and accumulator (O0 / O1 in TMEM), and the epilogue
+// merges the two row by row (all in log2 units):
+//   m = max(m0, m1), l = 2^(m0 - m) l0 + 2^(m1 - m) l1,
+//   O = (2^(m0 - m) O0 + 2^(m1 - m) O1) / l.
+// With a random block mask, two neighbouring query tiles seldom see the same
+// key tile, so the paired skipping form runs most of its iterations with one
+// live query tile; here both streams have a key tile in every iteration but
+// the last. The K/V ring holds L's tiles in list order (K then V of each),
+// each used by one stream only.
+template <int D>
+struct SCfg {
+  static constexpr int kSlots = (D == 64) ? 10 : 5;
+  static constexpr int kTileBytes = kBN * D * 2;
+  static constexpr int kQBytes = kBM * D * 2;
+  static constexpr int kColBlocks = D / 64;
+  static constexpr int kBlockBytes = 128 * 128;
+  static constexpr int kEmuPairs = Cfg<D, false>::kEmuPairs;
+  static constexpr uint32_t kS0 = 0, kS1 = 128;
+  static constexpr uint32_t kO0 = 256, kO1 = 256 + (D == 64 ? 64 : 128);
+  static constexpr uint32_t kPOff = 64;
+  static constexpr int kOffQ = 0;                  // also the O staging in the epilogue
+  static constexpr int kOffKV = kQBytes;
+  static constexpr int kOffEnd = kOffKV + kSlots * kTileBytes;
+  static_assert(kSlots <= kMaxSlots, "ring barriers");
+};
+
+struct CtlSplit : CtlCore {
+  uint16_t tiles[kMaxTiles];   // L: visible key tiles of the query tile, | kFullBit
+  float2 stat[2][kBM];         // per stream and row: (reference maximum, sum), log2 units
+};
+
+template <int D, bool kCap>
+__global__ void __launch_bounds__(kThreads, 1) fwd_split_kernel(const __grid_constant__ FwdParams p) {
+  using C = SCfg<D>;
+  constexpr int kSlots = C::kSlots;
+  extern __shared__ uint8_t smem_raw[];
+  CtlSplit& ctl = *reinterpret_cast<CtlSplit*>(smem_raw);
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t tile_addr = (raw_addr + sizeof(CtlSplit) + 1023u) & ~1023u;
+  uint8_t* tiles_base = smem_raw + (tile_addr - raw_addr);
+
+  // one query tile per CTA: heads p.chunk at a time, tiles from the last
+  int bh, rqb;
+  chunked_order(blockIdx.x, p.nb, p.BH, p.chunk, bh, rqb);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qb = p.nb - 1 - rqb;
+  const int h = bh % p.Hq, b = bh / p.Hq;
+  const int bhk = b * p.Hkv + h / (p.Hq / p.Hkv);
+  const int N = p.N, nb = p.nb;
+  const int q0 = qb * kBM;
+  const int kb_end = min(nb, mod_last_key(p.mod, q0 + kBM - 1, N) / kBN + 1);
+
+  if (threadIdx.x == 0) {
+    // (as in fwd_kernel: the error word is read once, and the CTA leaves
+    // together after the block barrier if it was set)
+    const unsigned err_word = *reinterpret_cast<volatile unsigned*>(p.err);
+    mbar_init(&ctl.q_full, 1);
+    for (int s = 0; s < kSlots; ++s) {
+      mbar_init(&ctl.kv_full[s], 1);
+      mbar_init(&ctl.kv_empty[s], 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&ctl.s_full[t], 1);
+      mbar_init(&ctl.p_half[t], 4);
+      mbar_init(&ctl.p_full[t], 4);
+      mbar_init(&ctl.o_ready[t], 1);
+    }
+    mbar_init(&ctl.o_done, 1);
+    mbar_init(&ctl.never, 1);
+    ctl.abort = 0;
+    fence_mbar_init();
+    prefetch_tmap(&p.tq);
+    prefetch_tmap(&p.tk);
+    prefetch_tmap(&p.tv);
+    mbar_expect_tx(&ctl.q_full, C::kQBytes);
+    for (int cb = 0; cb < C::kColBlocks; ++cb)
+      tma_load_3d(tiles_base + C::kOffQ + cb * C::kBlockBytes, &p.tq, &ctl.q_full, cb * 64, q0,
+                  bh);
+    ctl.skip = err_word != 0u;
+  }
+  if (warp == 2) {
+    tmem_alloc(&ctl.tmem_base, 512);
+    tmem_relinquish();
+  }
+  if (warp == 3) {
+    // L: the key tiles below kb_end this query tile sees (block mask, then
+    // the modifier's classification), flagged when wholly visible
+    int count = 0;
+    for (int kb0 = 0; kb0 < kb_end; kb0 += 32) {
+      const int kb = kb0 + lane;
+      int cls = kTileEmpty;
+      if (kb < kb_end && (!p.mask || p.mask[(size_t)qb * nb + kb]))
+        cls = mod_classify(p.mod, q0, q0 + kBM - 1, kb * kBN, kb * kBN + kBN - 1, N);
+      const bool act = cls != kTileEmpty;
+      const unsigned bal = __ballot_sync(0xffffffffu, act);
+      if (act)
+        ctl.tiles[count + __popc(bal & ((1u << lane) - 1u))] =
+            static_cast<uint16_t>(kb | (cls == kTileFull ? kFullBit : 0));
+      count += __popc(bal);
+    }
+    if (lane == 0) ctl.ntiles = count;
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = ctl.tmem_base;
+  if (ctl.skip) {
+    if (threadIdx.x == 0) drain_wait(&ctl.q_full, 0);
+    if (warp == 2) tmem_dealloc(tm, 512);
+    return;
+  }
+  const int T = ctl.ntiles;                  // |L|
+  const int T0 = (T + 1) / 2, T1 = T / 2;    // tiles of stream 0 and stream 1
+  const Guard g{&ctl.abort, p.err};
+  // list entry i (stream i & 1, its step i >> 1) is ring tiles 2i (K) and 2i + 1 (V)
+  auto key_tile = [&](int i) { return static_cast<int>(ctl.tiles[i] & ~kFullBit); };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      int issued = 0;
+      for (int n = 0; n < 2 * T; ++n) {
+        const int s = ring_slot<kSlots>(n);
+        if (n >= kSlots &&
+            !mbar_wait_ready_first(&ctl.kv_empty[s], ring_phase<kSlots>(n - kSlots), g))
+          break;
+        mbar_expect_tx(&ctl.kv_full[s], C::kTileBytes);
+        for (int cb = 0; cb < C::kColBlocks; ++cb)
+          tma_load_3d(tiles_base + C::kOffKV + s * C::kTileBytes + cb * C::kBlockBytes,
+                      (n & 1) ? &p.tv : &p.tk, &ctl.kv_full[s], cb * 64, key_tile(n >> 1) * kBN,
+                      bhk);
+        issued = n + 1;
+      }
+      drain_wait(&ctl.q_full, 0);
+      for (int s = 0; s < kSlots && s < issued; ++s) {
+        const int last = s + ((issued - 1 - s) / kSlots) * kSlots;
+        drain_wait(&ctl.kv_full[s], ring_phase<kSlots>(last));
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && T > 0) {
+      constexpr uint32_t idS = idesc_bf16(kBM, kBN, false, false);
+      constexpr uint32_t idO = idesc_bf16(kBM, D, false, true);
+      const uint64_t dq = sdesc_sw128(smem_u32(tiles_base + C::kOffQ), 16, 1024);
+      const uint64_t dk0 = sdesc_sw128(smem_u32(tiles_base + C::kOffKV), 16, 1024);
+      const uint64_t dv0 = sdesc_sw128(smem_u32(tiles_base + C::kOffKV), C::kBlockBytes, 1024);
+      auto wait_tile = [&](int n) {
+        return mbar_wait_ready_first(&ctl.kv_full[ring_slot<kSlots>(n)], ring_phase<kSlots>(n), g);
+      };
+      auto release_tile = [&](int n) { mma_commit(&ctl.kv_empty[ring_slot<kSlots>(n)]); };
+      // S_t = Q K^T for list entry i (stream t = i & 1), K the ring tile 2i
+      auto issue_s = [&](int i) {
+        const int t = i & 1;
+        const uint64_t dk = sdesc_at(dk0, ring_slot<kSlots>(2 * i) * C::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * C::kBlockBytes + (kk & 3) * 32;
+          mma_ss(tm + (t ? C::kS1 : C::kS0), sdesc_at(dq, off), sdesc_at(dk, off), idS, kk > 0);
+        }
+      };
+      // O_t += P_t V over keys 64*hf .. 64*hf+63, V the ring tile 2i + 1
+      auto issue_pv = [&](int i, bool acc, int hf) {
+        const int t = i & 1;
+        const uint64_t dv = sdesc_at(dv0, ring_slot<kSlots>(2 * i + 1) * C::kTileBytes);
+        const uint32_t pt = tm + (t ? C::kS1 : C::kS0) + C::kPOff;
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+          const int kk = 4 * hf + k4;
+          mma_ts(tm + (t ? C::kO1 : C::kO0), pt + kk * 8, sdesc_at(dv, kk * 16 * 128), idO,
+                 (acc || kk > 0));
+        }
+      };
+      bool ok = injected_stall(&ctl.never, p.stall, g) && mbar_wait_ready_first(&ctl.q_full, 0, g);
+      // the first S of each stream
+      for (int i = 0; ok && i < 2 && i < T; ++i) {
+        if (!(ok = wait_tile(2 * i))) break;
+        tc_fence_after();
+        issue_s(i);
+        mma_commit(&ctl.s_full[i]);
+        release_tile(2 * i);   // K of entry i
+      }
+      // step j: entry 2j of stream 0, entry 2j + 1 of stream 1 (if any)
+      for (int j = 0; ok && j < T0; ++j) {
+        for (int t = 0; t < 2; ++t) {
+          const int i = 2 * j + t;
+          if (i >= T) break;
+          const int nxt = i + 2;   // the stream's next entry
+          if (!(ok = wait_tile(2 * i + 1) && mbar_wait_ready_first(&ctl.p_half[t], j & 1, g)))
+            break;
+          tc_fence_after();
+          issue_pv(i, j > 0, 0);
+          if (!(ok = mbar_wait_ready_first(&ctl.p_full[t], j & 1, g))) break;
+          tc_fence_after();
+          issue_pv(i, j > 0, 1);
+          release_tile(2 * i + 1);   // V of entry i
+          if (nxt < T) {
+            // (its K is checked only now: with few ring slots it may still be
+            // loading, and stream 1's P V must not wait for it)
+            if (!(ok = wait_tile(2 * nxt))) break;
+            tc_fence_after();
+            issue_s(nxt);            // after P V in order: S overwrites P
+            mma_commit(&ctl.s_full[t]);
+            release_tile(2 * nxt);   // K of the next entry
+          } else {
+            mma_commit(&ctl.o_ready[t]);   // the stream's last P V
+          }
+        }
+      }
+      mma_commit(&ctl.o_done);
+      drain_wait(&ctl.o_done, 0);   // no MMA may still run when TMEM is freed
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------ softmax streams
+    const int t = (warp - 4) >> 2;           // stream of this warpgroup
+    const int wq = warp & 3;                 // TMEM lane quarter of this warp
+    const int r = wq * 32 + lane;            // row inside the query tile
+    const int row = q0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t sreg = tm + (t ? C::kS1 : C::kS0) + lane_off;
+    const float c = kCap ? 1.f : p.c;
+    const int Tt = t ? T1 : T0;
+    int row_lo, row_hi;
+    mod_row_keys(p.mod, row, N, row_lo, row_hi);
+    float m_ref = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < Tt; ++j) {
+      if (!(ok = mbar_wait_ready_first(&ctl.s_full[t], j & 1, g))) break;
+      tc_fence_after();
+      uint32_t sr[128];
+      tmem_ld128(sreg, sr);
+      if constexpr (kCap) {
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          sr[i] = __float_as_uint(p.cap1 * tanh_ex2(__uint_as_float(sr[i]) * p.cap2));
+      }
+      const int e = ctl.tiles[2 * j + t];
+      const int col0 = (e & ~kFullBit) * kBN;
+      const bool need_mask = !(e & kFullBit);
+      if (need_mask) {
+        const int lo = row_lo - col0, hi = row_hi - col0;
+#pragma unroll
+        for (int i = 0; i < 128; ++i)
+          if (i < lo || i > hi) sr[i] = __float_as_uint(-INFINITY);
+      }
+      softmax_tile<D, C::kEmuPairs>(sr, need_mask, c, j, m_ref, l, sreg, sreg + C::kPOff,
+                                    tm + (t ? C::kO1 : C::kO0) + lane_off, &ctl.p_half[t],
+                                    &ctl.p_full[t], lane);
+    }
+    // ------------------------------------------------------------ merge + epilogue
+    // The stream's accumulator is complete once its last P V has (all S
+    // MMAs, which read the Q buffer, came before it).
+    if (Tt > 0 && ok) {
+      mbar_wait_ready_first(&ctl.o_ready[t], 0, g);
+      tc_fence_after();
+    }
+    ctl.stat[t][r] = make_float2(Tt > 0 ? m_ref : -INFINITY, Tt > 0 ? l : 0.f);
+    named_sync(1, 256);
+    const float2 s0 = ctl.stat[0][r], s1 = ctl.stat[1][r];
+    const float m = fmaxf(s0.x, s1.x);
+    const float f0 = (s0.y > 0.f) ? ex2(s0.x - m) : 0.f;
+    const float f1 = (s1.y > 0.f) ? ex2(s1.x - m) : 0.f;
+    const float lsum = f0 * s0.y + f1 * s1.y;
+    const float inv = (lsum > 0.f) ? 1.f / lsum : 0.f;
+    const float w0 = f0 * inv, w1 = f1 * inv;
+    // this warpgroup writes columns [t * D/2, (t + 1) * D/2) of the row,
+    // from both streams' accumulators, into the Q buffer (128-byte swizzle)
+    uint8_t* stage = tiles_base + C::kOffQ;
+#pragma unroll
+    for (int cc = 0; cc < D / 64; ++cc) {
+      const int col = t * (D / 2) + cc * 32;     // first of 32 columns
+      uint32_t o0[32], o1[32];
+      if (T0 > 0) {
+        tmem_ld32(tm + C::kO0 + lane_off + col, o0);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o0[i] = 0u;
+      }
+      if (T1 > 0) {
+        tmem_ld32(tm + C::kO1 + lane_off + col, o1);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) o1[i] = 0u;
+      }
+      uint32_t w[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i)
+        w[i] = pack_bf16(fmaf(__uint_as_float(o0[2 * i]), w0, __uint_as_float(o1[2 * i]) * w1),
+                         fmaf(__uint_as_float(o0[2 * i + 1]), w0,
+                              __uint_as_float(o1[2 * i + 1]) * w1));
+      uint8_t* rowp = stage + (col >> 6) * 16384 + r * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int ch = ((col & 63) >> 3) + q;   // 16-byte chunk of the 128-byte row
+        *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) << 4)) =
+            make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+      }
+    }
+    if (t == 0 && row < N)
+      p.LSE[(size_t)bh * N + row] = (lsum > 0.f) ? (m + log2f(lsum)) * kLn2 : -INFINITY;
+    fence_async_smem();
+    named_sync(1, 256);
+    if (warp == 4 && lane == 0) {
+#pragma unroll
+      for (int cb = 0; cb < C::kColBlocks; ++cb)
+        tma_store_3d(&p.to, stage + cb * C::kBlockBytes, cb * 64, q0, bh);
+      bulk_commit();
+      bulk_wait_read0();   // the staging is read before the CTA exits
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 2) {
+    tc_fence_after();
+    tmem_dealloc(tm, 512);
+  }
+}
+
 // Dynamic shared memory of one form: control block, alignment slack, tiles.
 template <int D, bool kSkip>
 constexpr size_t smem_bytes() {
   return sizeof(Ctl<kSkip>) + 1024 + Cfg<D, kSkip>::kOffEnd;
+}
+template <int D>
+constexpr size_t split_smem_bytes() {
+  return sizeof(CtlSplit) + 1024 + SCfg<D>::kOffEnd;
 }
 template <int D>
 constexpr size_t persist_smem_bytes() {
@@ -1196,6 +1528,10 @@ cudaError_t launch(const Problem& pr) {
                          std::make_pair((const void*)fwd_kernel<D, false, true, true>, smem_skip),
                          std::make_pair((const void*)fwd_persist_kernel<D, false>,
                                         persist_smem_bytes<D>()),
+                         std::make_pair((const void*)fwd_split_kernel<D, false>,
+                                        split_smem_bytes<D>()),
+                         std::make_pair((const void*)fwd_split_kernel<D, true>,
+                                        split_smem_bytes<D>()),
                          std::make_pair((const void*)fwd_persist_kernel<D, true>,
                                         persist_smem_bytes<D>())}) {
     const cudaError_t e = set_max_dynamic_smem(fs.first, (int)fs.second);
@@ -1218,6 +1554,17 @@ cudaError_t launch(const Problem& pr) {
   const bool skip = !pr.cu && gaps;
   if (!skip && gaps) return cudaErrorInvalidValue;
   if (pr.cu && cap) return cudaErrorInvalidValue;   // not offered for packed batches
+  if (skip && pr.mask != nullptr && (FA_FWD_SPLIT & (D == 64 ? 1 : 2))) {
+    // block-sparse: one query tile per CTA, its key tiles split between the
+    // two softmax warpgroups
+    const dim3 sgrid((unsigned)(BHq * (uint64_t)pr.nb));
+    if (cap)
+      fwd_split_kernel<D, true><<<sgrid, kThreads, split_smem_bytes<D>(), pr.stream>>>(kp);
+    else
+      fwd_split_kernel<D, false><<<sgrid, kThreads, split_smem_bytes<D>(), pr.stream>>>(kp);
+    count_launch();
+    return cudaGetLastError();
+  }
   if (!pr.cu && !skip && pr.N <= FA_FWD_PERSIST_MAXN) {
     // one CTA per SM, each walking items blockIdx.x, blockIdx.x + gridDim.x, ...
     int dev = 0, sms = 0;
