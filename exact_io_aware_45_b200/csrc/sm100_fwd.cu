@@ -85,7 +85,8 @@ constexpr int kMaxSlots = 10;     // most K/V ring slots of any form
 // fixed cost per item matters most there) and 3-6% slower at 8K-16K (its
 // steady state is a little slower). 0: never persistent.
 // Block-sparse launches (a block mask given) run the split form: bit 0 at
-// d = 64, bit 1 at d = 128; otherwise the paired skipping form.
+// d = 64, bit 1 at d = 128; otherwise the paired skipping form. Bit 2: every
+// launch of the skipping form (windows, documents) runs the split form too.
 #ifndef FA_FWD_SPLIT
 #define FA_FWD_SPLIT 3
 #endif
@@ -1554,7 +1555,7 @@ cudaError_t launch(const Problem& pr) {
   const bool skip = !pr.cu && gaps;
   if (!skip && gaps) return cudaErrorInvalidValue;
   if (pr.cu && cap) return cudaErrorInvalidValue;   // not offered for packed batches
-  if (skip && pr.mask != nullptr && (FA_FWD_SPLIT & (D == 64 ? 1 : 2))) {
+  if (skip && (pr.mask != nullptr || (FA_FWD_SPLIT & 4)) && (FA_FWD_SPLIT & (D == 64 ? 1 : 2))) {
     // block-sparse: one query tile per CTA, its key tiles split between the
     // two softmax warpgroups
     const dim3 sgrid((unsigned)(BHq * (uint64_t)pr.nb));
