@@ -136,6 +136,9 @@ BLOCK_PATTERNS = {
     # every key tile is seen by exactly one tile of the first pair; the second
     # pair has one empty row and one row with a gap
     "alternating": [[1, 0, 1, 0], [0, 1, 0, 1], [0, 0, 0, 0], [1, 1, 0, 1]],
+    # query tiles that see exactly one key tile (one softmax stream of the
+    # split form has nothing), and one that sees all three
+    "single": [[1, 0, 0], [0, 0, 1], [1, 1, 1]],
 }
 
 
@@ -297,3 +300,21 @@ def test_autograd_attention(dt_name):
             assert_close_bf16(name, to_np(got), want)
         else:
             assert max_abs(to_np(got), want) <= 1e-4, name
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_block_mask_ragged(causal, d):
+    """Random block masks with a ragged last tile (N = 700): the split form's
+    last query tile has rows past N and its last key tile keys past N."""
+    x = inputs.random_case(1, 2, 1, 700, d, seed=23 + d + int(causal), mask_density=0.5)
+    scale = 1.0 / np.sqrt(d)
+    r = _run(x, scale, causal, fa.PATH_AUTO)
+    O, L = orc.forward(x["q"], x["k"], x["v"], scale, causal, x["mask"])
+    o, lse = to_np(r["o"]), to_np(r["lse"])
+    assert_close_bf16("O", o, O)
+    assert lse_err(lse, L) <= LSE_MAX_ABS
+    dQ, dK, dV = orc.backward(x["q"], x["k"], x["v"], x["do"], scale, causal, x["mask"], O=O)
+    assert_close_bf16("dQ", to_np(r["dq"]), dQ)
+    assert_close_bf16("dK", to_np(r["dk"]), dK)
+    assert_close_bf16("dV", to_np(r["dv"]), dV)
