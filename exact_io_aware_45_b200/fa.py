@@ -376,14 +376,15 @@ def backward_window(q, k, v, o, do, lse, window_left: int, window_right: int,
 
 
 def forward_mod(q, k, v, m: FaMods, scale: Optional[float] = None, causal: bool = False,
-                block_mask=None, workspace=None):
-    """O, LSE with mask modifiers (fa_fwd_mod); layouts as forward."""
+                block_mask=None, workspace=None, out=None, lse=None):
+    """O, LSE with mask modifiers (fa_fwd_mod); layouts and out / lse / workspace
+    as forward."""
     import torch
     B, Hq, Hkv, N, d = _dims(q, k)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    o = torch.empty_like(q)
-    l = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device)
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, Hq, N), dtype=torch.float32, device=q.device) if lse is None else lse
     ws = new_workspace(fa_fwd_workspace_size(), q.device) if workspace is None else workspace
     s = fa_fwd_mod(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(l), B, Hq, Hkv, N, d, float(scale),
                    int(bool(causal)), _ptr(block_mask), ctypes.byref(m), _dtype_code(q.dtype),
