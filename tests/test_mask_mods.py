@@ -33,6 +33,12 @@ CASES = [
     ("softcap", 1, 2, 1, 600, 128, False, None, 0, None, None, 1.5),
     ("softcap_causal_d64", 2, 2, 2, 300, 64, True, None, 0, None, None, 0.8),
     ("softcap_docs_mask", 1, 2, 1, 640, 64, True, (100, -1), 0, [300, 340], 0.5, 2.0),
+    # the capped variant of each remaining forward form: skipping (a left
+    # window edge, no block mask), split at d = 128 (a block mask), one-item
+    # (above the persistent form's 4,096 keys)
+    ("softcap_window_d128", 1, 2, 1, 640, 128, True, (150, -1), 0, [200, 440], None, 1.7),
+    ("softcap_mask_d128", 1, 2, 1, 520, 128, False, None, 0, None, 0.5, 1.0),
+    ("softcap_long_d64", 1, 1, 1, 4200, 64, True, None, 0, None, None, 1.2),
 ]
 
 
