@@ -36,11 +36,18 @@
 // a window edge, the causal diagonal of the other tile) is either computed for
 // it fully masked, keeping the two tiles in lockstep (dense, causal and
 // variable-length launches, where there are at most one or two such tiles per
-// CTA), or skipped for it: no Q K^T, softmax or P V (kSkip: block-sparse masks
-// and windows with a left edge, where a random mask makes about 40% of the
-// halves dead). The skipping form counts barrier phases per query tile;
-// measured on B200 it is 4-12% slower than the lockstep form where nearly
-// every tile is seen by both query tiles, hence the two forms.
+// CTA), or skipped for it: no Q K^T, softmax or P V (kSkip: windows with a
+// left edge and documents). The skipping form counts barrier phases per query
+// tile; measured on B200 it is 4-12% slower than the lockstep form where
+// nearly every tile is seen by both query tiles, hence the two forms.
+//
+// Forms per launch: the persistent form of the lockstep kernel (one CTA per
+// SM drawing two-tile items from a queue) for dense and causal launches up to
+// FA_FWD_PERSIST_MAXN keys; the one-item lockstep form above that and for
+// variable-length batches; the skipping form for left window edges and
+// documents; and, for block masks, the split form (one query tile per CTA,
+// its visible key tiles dealt to the two softmax warpgroups, the two partial
+// results merged by their log-sum-exp).
 //
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warp 2
 // TMEM allocator, warp 3 builds the key-tile list, warps 4-7 softmax of query
